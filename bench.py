@@ -1,0 +1,377 @@
+"""Benchmark of the NVFP4 W4A4 linear-layer hot path on B200.
+
+One step = one forward of the FLUX double-stream MLP-up layer
+(M=4608 tokens, K=3072, N=12288, bf16 bias): runtime NVFP4 quantization of
+the bf16 activations with the calibrated input scale, then the block-scaled
+NVFP4 GEMM with the fused alpha*acc + bias -> bf16 epilogue.  Inputs are
+seeded synthetic tensors of that shape (weights quantized once, untimed).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is whole-job TFLOP/s (2*M*N*K per
+step per GPU) with inputs resident in HBM; L2 is flushed between timed steps
+and every step is bracketed by CUDA events on the launching stream.  Under
+torchrun each rank runs its own token batch (weak scaling, no data
+collective); the step time is the max over ranks.
+``--impl reference`` times the CPU oracle on a bounded row sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GEMM TFLOP/s and % dense-FP4 peak; quantize GB/s and % HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PFLOP/s FP4 vs 2.25 PFLOP/s bf16
+QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
+
+    def summary(self, t0=None, t1=None):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((ts, float(parts[0]), float(parts[1]), parts))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        inside = [r for r in rows if t0 is None or (t0 <= r[0] <= t1)] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, _, parts in inside:
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle
+ORACLE_COLS = 1024  # weight rows (output columns) in the oracle's sample block
+
+
+def oracle_sample(rows: int, step: int = 0):
+    """Time the oracle on a block of the MLP-up layer: `rows` activation rows
+    (a different slice each step) x ORACLE_COLS output columns.  Timed: the
+    runtime activation quantize of those rows and the fp64
+    dequantize-then-matmul + bias.  The weight block is quantized once,
+    untimed (weight preparation is offline).  Returns (seconds, flops)."""
+    import oracle as O
+    import synth
+    wl = synth.MLP_UP
+    x = synth_cache("x", lambda: wl.activations().float().numpy())
+    gx = synth_cache("gx", lambda: O.global_scale(O.tensor_amax(x)))
+    wq = synth_cache("wq", lambda: _oracle_weight(O, wl))
+    bias = synth_cache("bias", lambda: wl.bias_vec().float().numpy()[:ORACLE_COLS])
+    r0 = (step * rows) % (wl.m - rows + 1)
+    t0 = time.perf_counter()
+    xc, xs = O.quantize_nvfp4(x[r0:r0 + rows], gx)
+    O.gemm_ref(xc, xs, gx, wq[0], wq[1], wq[2], bias)
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * rows * ORACLE_COLS * wl.k
+
+
+_CACHE = {}
+
+
+def synth_cache(key, fn):
+    if key not in _CACHE:
+        _CACHE[key] = fn()
+    return _CACHE[key]
+
+
+def _oracle_weight(O, wl):
+    w = wl.weight().float().numpy()
+    gw = O.global_scale(O.tensor_amax(w))  # per-tensor scale over the whole weight
+    wc, ws = O.quantize_nvfp4(w[:ORACLE_COLS], gw)
+    return wc, ws, gw
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i.get("num_threads", 0)) for i in threadpool_info()]
+        return max(n) if n else os.cpu_count() or 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float = 10.0, rows: int = 256):
+    """The oracle as it stands, on a bounded sample of the workload."""
+    oracle_sample(8)  # build the cached inputs (untimed)
+    total_t, total_f, n = 0.0, 0.0, 0
+    while total_t < budget_s and n < 400:
+        dt, fl = oracle_sample(rows, n)
+        total_t += dt
+        total_f += fl
+        n += 1
+    return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} blocks of {rows} activation rows x {ORACLE_COLS} output columns of "
+                      f"M=4608,K=3072,N=12288 (quantize + fp64 GEMM + bias), {total_t:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    rows = 128
+    oracle_sample(8)  # build the cached inputs (untimed)
+    for i in range(args.warmup):
+        oracle_sample(rows, i)
+    times, flops = [], 0.0
+    for i in range(args.steps):
+        dt, fl = oracle_sample(rows, args.warmup + i)
+        times.append(dt)
+        flops += fl
+    tot = sum(times)
+    val = flops / tot / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "flux_mlp_up_m4608_k3072_n12288", "m": 4608, "k": 3072, "n": 12288,
+                   "step_sample_rows": rows, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{rows} activation rows x {ORACLE_COLS} output columns per step of "
+                                   "M=4608,K=3072,N=12288"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import nvfp4_block_scaled_12_b200 as F
+    import synth
+
+    wl = synth.MLP_UP
+    M, K, N = wl.m, wl.k, wl.n
+    flops = 2.0 * M * N * K
+    # each rank gets its own token batch (independent seeds): weak scaling
+    x = synth.activations_with_outlier_channels(M, K, seed=wl.seed + 100 * rank).to(device)
+    w = wl.weight().to(device)
+    bias = wl.bias_vec().to(device)
+    g_x = F.global_scale(x)              # calibrated input_scale (offline)
+    wq = F.quantize(w, F.global_scale(w))  # ModelOpt-style weight prep (offline)
+    xq = F.quantize(x, g_x)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        F.quantize(x, g_x, out=xq, stream=stream)
+        F.gemm(xq, wq, bias=bias, y=y, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    F.nvfp4_check_fault()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local if not os.environ.get("CUDA_VISIBLE_DEVICES") else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    sampler.start()
+    time.sleep(0.2)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps, outside the events
+        ev[i][0].record(stream)
+        F.quantize(x, g_x, out=xq, stream=stream)
+        ev[i][1].record(stream)
+        F.gemm(xq, wq, bias=bias, y=y, stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(device)
+    t_wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    F.nvfp4_check_fault()
+
+    q_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    g_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    step_ms = sum(q_ms) / args.steps + sum(g_ms) / args.steps
+    step_ms_max = max_over_ranks(step_ms, world, device)
+    gemm_ms = max_over_ranks(sum(g_ms) / args.steps, world, device)
+    quant_ms = max_over_ranks(sum(q_ms) / args.steps, world, device)
+
+    # end to end through the public API with host buffers: pinned x in,
+    # pinned y out, copies inside the timed region
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        F.quantize(x_dev, g_x, out=xq, stream=stream)
+        F.gemm(xq, wq, bias=bias, y=y, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        F.quantize(x_dev, g_x, out=xq, stream=stream)
+        F.gemm(xq, wq, bias=bias, y=y, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
+
+    if rank == 0:
+        hbm, bf16, src = peaks()
+        fp4_peak = bf16 * FP4_PER_BF16
+        gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
+        quant_gbs = M * K * QUANT_BYTES_PER_ELEM / (quant_ms * 1e-3) / 1e9
+        clocks = sampler.summary(t_wall0, t_wall1)
+        line = {
+            "metric": METRIC,
+            "value": world * flops / (step_ms_max * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": step_ms_max,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "fp4(e2m1)xfp4->f32 accum, bf16 out",
+            "data": "synthetic",
+            "config": {"workload": "flux_mlp_up_m4608_k3072_n12288", "m": M, "k": K, "n": N,
+                       "bias": True, "global_batch_tokens": world * M, "parallelism": f"dp{world} (token shards)",
+                       "l2": "flushed between timed steps (256 MiB write)"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tf / fp4_peak, "traffic": None,
+                         "peak_source": f"{src} bf16 burst x {FP4_PER_BF16:g} (nominal FP4/bf16 dense ratio)"},
+            "kernels": {
+                "gemm": {"ms": gemm_ms, "tflops": gemm_tf, "frac_of_fp4_peak": gemm_tf / fp4_peak},
+                "quantize": {"ms": quant_ms, "gbs": quant_gbs, "frac_of_hbm": quant_gbs / hbm,
+                             "bytes": M * K * QUANT_BYTES_PER_ELEM, "hbm_peak_gbs": hbm, "peak_source": src},
+            },
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+            "gpu_launches": 2 * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+                       "samples": clocks["samples"]},
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

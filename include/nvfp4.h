@@ -1,0 +1,200 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 W4A4 linear-layer library.
+ *
+ * The operation: an NVFP4 linear layer as run on Blackwell, i.e. runtime
+ * quantization of bf16 activations to NVFP4 followed by an NVFP4 x NVFP4
+ * block-scaled GEMM against ModelOpt-layout weights ("BFL (fp8r / nvfp4)"
+ * diffusers doc, section "Kernels", table row `nvfp4`: `nvfp4_quantize` on the
+ * activations, `mm_fp4` for the GEMM).
+ *
+ * NVFP4 format ("NVIDIA FP4 format" news page, paragraph 1; BFL doc, `nvfp4`
+ * bullet): 4-bit E2M1 elements, two per byte, one E4M3 scale per 16 elements
+ * along K, plus one fp32 per-tensor scale.  This library uses the DECODE
+ * convention for the per-tensor scale everywhere:
+ *     x_hat = e2m1(code) * e4m3(block_scale) * g,   g = amax / (6 * 448)
+ * so g is ModelOpt's `input_scale` for activations and `weight_scale_2` for
+ * weights, and the GEMM's alpha is input_scale * weight_scale_2.
+ *
+ * Layouts (all row-major, all buffers owned by the caller):
+ *   bf16 activations  x      [M, K]      2 bytes/elem
+ *   codes             q      [rows, K/2] uint8; element 2j in bits 0-3 of
+ *                                        byte j, element 2j+1 in bits 4-7
+ *   linear scales            [rows, K/16] uint8 E4M3 (ModelOpt `weight_scale`)
+ *   swizzled scales          nvfp4_sf_bytes(rows, K) bytes: rows padded to a
+ *                            multiple of 128, scale columns (K/16) padded to a
+ *                            multiple of 4, cut into 512-byte atoms of
+ *                            128 rows x 4 scale columns stored atom-row-major;
+ *                            logical (r, c) sits at byte
+ *         ((r/128)*(Cp/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4
+ *                            with Cp = padded scale columns.  Padding is 0.
+ *                            This is the layout the tcgen05 block-scaled MMA
+ *                            reads scale factors in.
+ *   bf16 output       y      [M, N]  (GEMM; B is the weight [N, K], i.e.
+ *                                     PyTorch's [out_features, in_features])
+ *
+ * Common contract of every entry point:
+ *   - Pointers are device pointers on the current CUDA device, 16-byte
+ *     aligned, unless stated otherwise.  The library allocates nothing and
+ *     keeps no state besides per-device caches (device properties, the
+ *     address of its device fault word).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: a return of NVFP4_OK means the work was
+ *     validated and launched, not that it finished.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call launches nothing and returns a non-zero status with a
+ *     message available from nvfp4_last_error() (thread-local).
+ *   - The current device must be compute capability 10.0 (B200, sm_100a);
+ *     otherwise NVFP4_EARCH.  There is no CPU fallback.
+ *   - K is a multiple of 64 and at least 64.
+ *   - Per-tensor scales (g, alpha) must be finite; g must lie in
+ *     [2^-64, 2^64] so that no intermediate of the quantizer overflows.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_EINVAL = 1,   /* bad size, null pointer, bad scale or range list   */
+  NVFP4_EALIGN = 2,   /* a pointer or leading dimension is misaligned     */
+  NVFP4_EARCH = 3,    /* current device is not compute capability 10.0    */
+  NVFP4_ECUDA = 4,    /* a CUDA runtime / driver call or launch failed     */
+  NVFP4_ETIMEOUT = 5  /* a kernel gave up waiting on one of its barriers   */
+} nvfp4_status;
+
+/* Activation applied by the fused epilogue to a column range. */
+enum { NVFP4_ACT_NONE = 0, NVFP4_ACT_GELU_TANH = 1 };
+/* Destination of a column range in the fused epilogue. */
+enum { NVFP4_DST_BF16 = 0, NVFP4_DST_NVFP4 = 1 };
+
+/* Most column ranges nvfp4_gemm_quant accepts. */
+#define NVFP4_MAX_RANGES 8
+
+/*
+ * Size in bytes of the swizzled scale buffer for a [rows, k] NVFP4 tensor:
+ * ceil(rows/128)*128 * ceil(k/64)*4.  Returns 0 if rows < 1 or k < 16 or
+ * k % 16 != 0.  Host-only, no CUDA call.
+ */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
+
+/*
+ * Per-tensor scale calibration (BFL doc, `nvfp4` bullet: the calibrated fp32
+ * `input_scale` and the global fp32 `weight_scale_2`):
+ *     out[0] = amax = max |x_i| over the n bf16 values (exact)
+ *     out[1] = g    = fl(amax / 2688)          (2688 = 6 * 448)
+ * x is [n] bf16 with n % 8 == 0, n >= 8; out is 2 device floats (8 bytes,
+ * 4-byte aligned), written.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_calibrate(const void* x, int64_t n, float* out, void* stream);
+
+/*
+ * Runtime activation quantization, bf16 -> NVFP4 (BFL doc, "Kernels",
+ * `nvfp4_quantize`).  For each row and each 16-element block along K, with
+ * every step one IEEE fp32 operation rounded to nearest even:
+ *     amax = max |x_i|;  s = E4M3_satfinite(amax / (6*g))
+ *     s == 0  ->  all 16 codes 0x0
+ *     else       r = 1 / (e4m3(s) * g);  code_i = E2M1_satfinite(x_i * r)
+ * E2M1 rounding is to nearest, ties to the even code, saturating at +-6; the
+ * code's sign bit is the sign of x_i * r (so -0 inputs give 0x8).  E4M3 never
+ * produces NaN (saturates at 448).
+ *   x      [M, K] bf16, read only.
+ *   g      per-tensor decode scale (calibrated input_scale), in [2^-64, 2^64].
+ *   codes  [M, K/2] uint8, written.
+ *   sf     nvfp4_sf_bytes(M, K) bytes, written in the swizzled layout,
+ *          including its zero padding rows.
+ * M >= 1.  Errors: EINVAL (sizes, null, g), EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g,
+                            uint8_t* codes, uint8_t* sf, void* stream);
+
+/*
+ * Weight preparation: scatter ModelOpt's row-major E4M3 `weight_scale`
+ * [rows, k/16] into the swizzled layout the GEMM reads (a byte permutation;
+ * padding bytes are written as 0).  sf_linear needs no alignment;
+ * sf_swizzled (nvfp4_sf_bytes(rows, k) bytes) must be 16-byte aligned.
+ * rows >= 1, k % 64 == 0.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_swizzle_sf(const uint8_t* sf_linear, int64_t rows, int64_t k,
+                              uint8_t* sf_swizzled, void* stream);
+
+/*
+ * Block-scaled NVFP4 GEMM with the dequant folded into the epilogue
+ * (BFL doc, "Kernels", `mm_fp4`):
+ *     y[m, n] = bf16_rn( alpha * sum_k a_hat[m,k] * b_hat[n,k] + bias[n] )
+ * with a_hat = e2m1(a) * e4m3(sfa) and b_hat likewise; the sum is
+ * accumulated in fp32 by the tensor cores (tcgen05, kind::mxf4nvf4, one
+ * E4M3 scale per 16 elements).
+ *   a     [M, K/2] codes (activations), sfa swizzled nvfp4_sf_bytes(M, K)
+ *   b     [N, K/2] codes (weights),     sfb swizzled nvfp4_sf_bytes(N, K)
+ *   alpha input_scale * weight_scale_2 (finite)
+ *   bias  [N] bf16 or NULL
+ *   y     [M, N] bf16, written
+ * M >= 1, N >= 8 with N % 8 == 0.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ * A barrier wait inside the kernel that exceeds its time limit makes the
+ * kernel return early and record NVFP4_ETIMEOUT in the device fault word
+ * (see nvfp4_check_fault).
+ */
+nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                        const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                        float alpha, const void* bias, void* y, void* stream);
+
+/* One column range of the fused epilogue. */
+typedef struct nvfp4_colrange {
+  int64_t begin;   /* first GEMM output column of the range              */
+  int64_t end;     /* one past the last column                           */
+  int32_t act;     /* NVFP4_ACT_NONE or NVFP4_ACT_GELU_TANH              */
+  int32_t dst;     /* NVFP4_DST_BF16 or NVFP4_DST_NVFP4                  */
+  int64_t dst_col; /* first column written in the destination tensor     */
+} nvfp4_colrange;
+
+/*
+ * GEMM with a fused epilogue that writes the next layer's input.  For every
+ * output column n in range i:
+ *     v = bf16_rn(alpha * acc[m,n] + bias[n])
+ *     if act == GELU_TANH:  v = bf16_rn(gelu_tanh(v))
+ *       (0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), fp32)
+ *     dst == BF16:   y_bf16[m, dst_col + n - begin] = v
+ *     dst == NVFP4:  v (bf16) is quantized exactly as nvfp4_quantize does,
+ *                    with scale g_next, into column dst_col + n - begin of
+ *                    the [M, k_next] NVFP4 tensor (codes_next, sf_next).
+ * Columns outside every range are dropped.  Ranges must not overlap; at most
+ * NVFP4_MAX_RANGES; begin, end and dst_col multiples of 64; end <= N;
+ * dst_col + (end - begin) <= ldy (BF16) or <= k_next (NVFP4).  The NVFP4
+ * destination's scale padding rows are written as zero; its scale columns
+ * belonging to no range are left untouched.
+ *   y_bf16     [M, ldy] bf16 (NULL if no BF16 range), ldy % 8 == 0
+ *   codes_next [M, k_next/2] uint8, sf_next nvfp4_sf_bytes(M, k_next)
+ *              (NULL if no NVFP4 range), k_next % 64 == 0
+ * Other arguments as nvfp4_gemm.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                              const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                              float alpha, const void* bias,
+                              const nvfp4_colrange* ranges, int32_t n_ranges,
+                              void* y_bf16, int64_t ldy,
+                              float g_next, uint8_t* codes_next, uint8_t* sf_next,
+                              int64_t k_next, void* stream);
+
+/*
+ * Synchronize the current device, then read and clear its fault word.
+ * Returns NVFP4_ETIMEOUT if any kernel of this library gave up on a barrier
+ * wait since the last check, NVFP4_ECUDA if the synchronize failed, else
+ * NVFP4_OK.
+ */
+nvfp4_status nvfp4_check_fault(void);
+
+/* Message describing the last error of the calling thread ("" if none).
+ * The pointer stays valid until the thread's next call into the library. */
+const char* nvfp4_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

@@ -1,0 +1,237 @@
+"""B200-native NVFP4 W4A4 linear layers: Python binding of ``libnvfp4.so``.
+
+The functions named ``nvfp4_*`` mirror the C ABI of ``include/nvfp4.h`` one to
+one (raw device pointers as ints, sizes, scales, a CUDA stream handle) and do
+argument marshalling only.  The helpers without the prefix (``quantize``,
+``gemm``, ``gemm_quant``, ``swizzle_sf``) take torch tensors, allocate the
+outputs with torch (device memory is the only thing torch provides here) and
+call the same entry points on the current torch stream.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback: the
+first call raises ImportError if the library was not built.
+
+Build the library with ``python -m nvfp4_block_scaled_12_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
+
+NVFP4_OK, NVFP4_EINVAL, NVFP4_EALIGN, NVFP4_EARCH, NVFP4_ECUDA, NVFP4_ETIMEOUT = range(6)
+ACT_NONE, ACT_GELU_TANH = 0, 1
+DST_BF16, DST_NVFP4 = 0, 1
+MAX_RANGES = 8
+
+_STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_EINVAL", 2: "NVFP4_EALIGN", 3: "NVFP4_EARCH", 4: "NVFP4_ECUDA",
+                 5: "NVFP4_ETIMEOUT"}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class ColRange(ctypes.Structure):
+    """``nvfp4_colrange``: one column range of the fused epilogue."""
+    _fields_ = [("begin", ctypes.c_int64), ("end", ctypes.c_int64), ("act", ctypes.c_int32),
+                ("dst", ctypes.c_int32), ("dst_col", ctypes.c_int64)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m nvfp4_block_scaled_12_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, f32, vp, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_int32
+    lib.nvfp4_sf_bytes.argtypes = [i64, i64]
+    lib.nvfp4_sf_bytes.restype = ctypes.c_size_t
+    lib.nvfp4_calibrate.argtypes = [vp, i64, vp, vp]
+    lib.nvfp4_quantize.argtypes = [vp, i64, i64, f32, vp, vp, vp]
+    lib.nvfp4_swizzle_sf.argtypes = [vp, i64, i64, vp, vp]
+    lib.nvfp4_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
+    lib.nvfp4_gemm_quant.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, ctypes.POINTER(ColRange), i32,
+                                     vp, i64, f32, vp, vp, i64, vp]
+    lib.nvfp4_check_fault.argtypes = []
+    for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant", "nvfp4_check_fault"):
+        getattr(lib, name).restype = ctypes.c_int
+    lib.nvfp4_last_error.argtypes = []
+    lib.nvfp4_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+_lib_handle: Optional[ctypes.CDLL] = None
+
+
+def library() -> ctypes.CDLL:
+    """The loaded ``libnvfp4.so`` (loaded on first use)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load()
+    return _lib_handle
+
+
+def _check(status: int) -> None:
+    if status != NVFP4_OK:
+        raise NVFP4Error(status, nvfp4_last_error())
+
+
+# --------------------------------------------------------------------------
+# 1:1 mirrors of the C ABI (pointers and streams as ints; 0 = NULL)
+# --------------------------------------------------------------------------
+
+def nvfp4_sf_bytes(rows: int, k: int) -> int:
+    return int(library().nvfp4_sf_bytes(rows, k))
+
+
+def nvfp4_calibrate(x: int, n: int, out: int, stream: int) -> None:
+    _check(library().nvfp4_calibrate(x, n, out, stream))
+
+
+def nvfp4_quantize(x: int, M: int, K: int, g: float, codes: int, sf: int, stream: int) -> None:
+    _check(library().nvfp4_quantize(x, M, K, g, codes, sf, stream))
+
+
+def nvfp4_swizzle_sf(sf_linear: int, rows: int, k: int, sf_swizzled: int, stream: int) -> None:
+    _check(library().nvfp4_swizzle_sf(sf_linear, rows, k, sf_swizzled, stream))
+
+
+def nvfp4_gemm(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha: float, bias: int, y: int,
+               stream: int) -> None:
+    _check(library().nvfp4_gemm(a, sfa, b, sfb, M, N, K, alpha, bias or None, y, stream))
+
+
+def nvfp4_gemm_quant(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha: float, bias: int,
+                     ranges: Sequence[ColRange], y_bf16: int, ldy: int, g_next: float, codes_next: int,
+                     sf_next: int, k_next: int, stream: int) -> None:
+    arr = (ColRange * len(ranges))(*ranges)
+    _check(library().nvfp4_gemm_quant(a, sfa, b, sfb, M, N, K, alpha, bias or None, arr, len(ranges), y_bf16 or None,
+                                 ldy, g_next, codes_next or None, sf_next or None, k_next, stream))
+
+
+def nvfp4_check_fault() -> None:
+    _check(library().nvfp4_check_fault())
+
+
+def nvfp4_last_error() -> str:
+    return library().nvfp4_last_error().decode()
+
+
+# --------------------------------------------------------------------------
+# torch-tensor helpers (outputs allocated with torch on the input's device)
+# --------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _need(t, dtype, shape, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class NVFP4Tensor:
+    """A [rows, k] NVFP4 tensor on the GPU: packed codes, swizzled scales and
+    the per-tensor decode scale g."""
+    codes: "object"   # uint8 [rows, k/2]
+    sf: "object"      # uint8 [nvfp4_sf_bytes(rows, k)]
+    g: float
+    rows: int
+    k: int
+
+
+def calibrate(x, stream=None):
+    """Per-tensor scale of bf16 ``x`` on the GPU.  Returns a float32 CUDA
+    tensor [amax, g] with g = amax / 2688 (nothing is read back)."""
+    torch = _torch()
+    _need(x, torch.bfloat16, None, "x")
+    out = torch.empty(2, dtype=torch.float32, device=x.device)
+    nvfp4_calibrate(_ptr(x), x.numel(), _ptr(out), _stream(stream))
+    return out
+
+
+def global_scale(x, stream=None) -> float:
+    """g = amax(|x|) / 2688 computed on the GPU, read back as a Python float."""
+    return float(calibrate(x, stream)[1].item())
+
+
+def quantize(x, g: float, out: Optional[NVFP4Tensor] = None, stream=None) -> NVFP4Tensor:
+    """Quantize bf16 ``x`` [M, K] to NVFP4 with per-tensor decode scale g."""
+    torch = _torch()
+    M, K = x.shape
+    _need(x, torch.bfloat16, None, "x")
+    if out is None:
+        out = NVFP4Tensor(torch.empty(M, K // 2, dtype=torch.uint8, device=x.device),
+                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=x.device), float(g), M, K)
+    nvfp4_quantize(_ptr(x), M, K, float(g), _ptr(out.codes), _ptr(out.sf), _stream(stream))
+    out.g = float(g)
+    return out
+
+
+def swizzle_sf(sf_linear, rows: int, k: int, stream=None):
+    """ModelOpt row-major E4M3 scales [rows, k/16] -> swizzled buffer."""
+    torch = _torch()
+    _need(sf_linear, torch.uint8, (rows, k // 16), "sf_linear")
+    out = torch.empty(nvfp4_sf_bytes(rows, k), dtype=torch.uint8, device=sf_linear.device)
+    nvfp4_swizzle_sf(_ptr(sf_linear), rows, k, _ptr(out), _stream(stream))
+    return out
+
+
+def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = None, y=None, stream=None):
+    """y = bf16(alpha * a_hat @ b_hat^T + bias); alpha defaults to fl32(a.g * b.g)."""
+    torch = _torch()
+    import numpy as np
+    if a.k != b.k:
+        raise ValueError("K mismatch")
+    M, N, K = a.rows, b.rows, a.k
+    if alpha is None:
+        alpha = float(np.float32(a.g) * np.float32(b.g))
+    if bias is not None:
+        _need(bias, torch.bfloat16, (N,), "bias")
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias), _ptr(y),
+               _stream(stream))
+    return y
+
+
+def gemm_quant(a: NVFP4Tensor, b: NVFP4Tensor, ranges: Sequence[tuple], *, bias=None, alpha=None, y_bf16=None,
+               g_next: float = 1.0, next_out: Optional[NVFP4Tensor] = None, stream=None) -> None:
+    """Fused GEMM whose epilogue writes column ranges to a bf16 tensor and/or
+    quantizes them into the next layer's NVFP4 input.  ``ranges`` holds
+    ``(begin, end, act, dst, dst_col)`` tuples."""
+    import numpy as np
+    M, N, K = a.rows, b.rows, a.k
+    if alpha is None:
+        alpha = float(np.float32(a.g) * np.float32(b.g))
+    rs = [ColRange(int(r[0]), int(r[1]), int(r[2]), int(r[3]), int(r[4])) for r in ranges]
+    ldy = int(y_bf16.shape[1]) if y_bf16 is not None else 0
+    codes_next = next_out.codes if next_out is not None else None
+    sf_next = next_out.sf if next_out is not None else None
+    k_next = next_out.k if next_out is not None else 0
+    nvfp4_gemm_quant(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias), rs,
+                     _ptr(y_bf16), ldy, float(g_next), _ptr(codes_next), _ptr(sf_next), k_next, _stream(stream))
+    if next_out is not None:
+        next_out.g = float(g_next)

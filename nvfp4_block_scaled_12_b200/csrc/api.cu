@@ -1,0 +1,325 @@
+// The library's C ABI (declared in include/nvfp4.h): argument validation,
+// device checks, TMA descriptor construction and kernel launch.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+
+namespace nvfp4 {
+
+int gemm_tile_n();
+
+namespace {
+
+// Fault word: kernels OR a code in here when a barrier wait times out.
+__device__ unsigned int g_fault_word;
+
+thread_local std::string t_last_error;
+
+nvfp4_status fail(nvfp4_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+nvfp4_status fail(nvfp4_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+nvfp4_status ok() {
+  t_last_error.clear();
+  return NVFP4_OK;
+}
+
+nvfp4_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(NVFP4_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+// Properties of the current device (cached); EARCH unless it is cc 10.0.
+nvfp4_status current_device(const DeviceInfo** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4_ECUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (d.device != dev) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    DeviceInfo n;
+    n.device = dev;
+    n.num_sms = prop.multiProcessorCount;
+    n.cc_major = prop.major;
+    n.cc_minor = prop.minor;
+    n.max_smem_optin = prop.sharedMemPerBlockOptin;
+    if (n.cc_major == 10 && n.cc_minor == 0) {
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, g_fault_word);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fault word)");
+      n.fault = static_cast<unsigned*>(addr);
+    }
+    d = n;
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0)
+    return fail(NVFP4_EARCH, "device %d has compute capability %d.%d; this library is built for 10.0 (sm_100a)",
+                dev, d.cc_major, d.cc_minor);
+  *out = &d;
+  return NVFP4_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with rows `row_bytes` apart.
+nvfp4_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw,
+                       const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(NVFP4_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ECUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
+  return NVFP4_OK;
+}
+
+bool finite_f(float v) { return isfinite(v) != 0; }
+
+bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
+
+// Checks shared by the two GEMM entry points; fills the operand part of p.
+nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
+                         int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, CUtensorMap* ta,
+                         CUtensorMap* tb, const DeviceInfo** dev) {
+  if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
+  if (M < 1 || M > INT32_MAX / 2) return fail(NVFP4_EINVAL, "M=%lld out of range", (long long)M);
+  if (N < 8 || N % 8 != 0 || N > INT32_MAX / 2)
+    return fail(NVFP4_EINVAL, "N=%lld must be a positive multiple of 8", (long long)N);
+  if (K < 64 || K % 64 != 0 || K > INT32_MAX / 2)
+    return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (!finite_f(alpha)) return fail(NVFP4_EINVAL, "alpha must be finite");
+  if (!aligned16(a) || !aligned16(sfa) || !aligned16(b) || !aligned16(sfb) || !aligned16(bias))
+    return fail(NVFP4_EALIGN, "operand pointers must be 16-byte aligned");
+  nvfp4_status st = current_device(dev);
+  if (st != NVFP4_OK) return st;
+
+  const int bn = gemm_tile_n();
+  *p = GemmParams{};
+  p->M = static_cast<int32_t>(M);
+  p->N = static_cast<int32_t>(N);
+  p->K = static_cast<int32_t>(K);
+  p->tiles_m = static_cast<int32_t>((M + 127) / 128);
+  p->tiles_n = static_cast<int32_t>((N + bn - 1) / bn);
+  const int64_t tiles = static_cast<int64_t>(p->tiles_m) * p->tiles_n;
+  if (tiles > INT32_MAX) return fail(NVFP4_EINVAL, "problem too large");
+  p->num_tiles = static_cast<int32_t>(tiles);
+  p->num_kt = static_cast<int32_t>((K + 255) / 256);
+  p->k64 = static_cast<int32_t>(K / 64);
+  p->sfb_row_blocks = static_cast<int32_t>((N + 127) / 128);
+  p->sfa = sfa;
+  p->sfb = sfb;
+  p->alpha = alpha;
+  p->bias = static_cast<const __nv_bfloat16*>(bias);
+  p->fault = (*dev)->fault;
+
+  st = make_tmap(ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+  if (st != NVFP4_OK) return st;
+  st = make_tmap(tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, bn, CU_TENSOR_MAP_SWIZZLE_128B, "B");
+  return st;
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k) {
+  if (rows < 1 || k < 16 || k % 16 != 0) return 0;
+  const int64_t rp = (rows + 127) / 128 * 128;
+  const int64_t cp = (k / 16 + 3) / 4 * 4;
+  return static_cast<size_t>(rp) * static_cast<size_t>(cp);
+}
+
+nvfp4_status nvfp4_calibrate(const void* x, int64_t n, float* out, void* stream) {
+  if (!x || !out) return fail(NVFP4_EINVAL, "null pointer");
+  if (n < 8 || n % 8 != 0) return fail(NVFP4_EINVAL, "n=%lld must be a positive multiple of 8", (long long)n);
+  if (!aligned16(x)) return fail(NVFP4_EALIGN, "x must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(out) & 3u) != 0) return fail(NVFP4_EALIGN, "out must be 4-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_calibrate(x, n, out, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "calibrate launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
+                            void* stream) {
+  if (!x || !codes || !sf) return fail(NVFP4_EINVAL, "null pointer");
+  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
+  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (!scale_ok(g)) return fail(NVFP4_EINVAL, "g=%g must be finite and in [2^-64, 2^64]", (double)g);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_quantize(x, M, K, g, codes, sf, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_swizzle_sf(const uint8_t* sf_linear, int64_t rows, int64_t k, uint8_t* sf_swizzled,
+                              void* stream) {
+  if (!sf_linear || !sf_swizzled) return fail(NVFP4_EINVAL, "null pointer");
+  if (rows < 1) return fail(NVFP4_EINVAL, "rows=%lld must be >= 1", (long long)rows);
+  if (k < 64 || k % 64 != 0) return fail(NVFP4_EINVAL, "k=%lld must be a positive multiple of 64", (long long)k);
+  if (!aligned16(sf_swizzled)) return fail(NVFP4_EALIGN, "sf_swizzled must be 16-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_swizzle_sf(sf_linear, rows, k, sf_swizzled, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "swizzle launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
+                        int64_t N, int64_t K, float alpha, const void* bias, void* y, void* stream) {
+  if (!y) return fail(NVFP4_EINVAL, "null output pointer");
+  if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
+  GemmParams p;
+  CUtensorMap ta, tb, ty;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &ta, &tb, &dev);
+  if (st != NVFP4_OK) return st;
+  st = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm(ta, tb, ty, p, false, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                              int64_t M, int64_t N, int64_t K, float alpha, const void* bias,
+                              const nvfp4_colrange* ranges, int32_t n_ranges, void* y_bf16, int64_t ldy,
+                              float g_next, uint8_t* codes_next, uint8_t* sf_next, int64_t k_next, void* stream) {
+  if (!ranges || n_ranges < 1 || n_ranges > NVFP4_MAX_RANGES)
+    return fail(NVFP4_EINVAL, "n_ranges=%d must be in [1, %d]", n_ranges, NVFP4_MAX_RANGES);
+  bool any_bf16 = false, any_fp4 = false;
+  for (int i = 0; i < n_ranges; ++i) {
+    const nvfp4_colrange& r = ranges[i];
+    if (r.begin < 0 || r.end <= r.begin || r.end > N || r.begin % 64 || r.end % 64 || r.dst_col < 0 ||
+        r.dst_col % 64)
+      return fail(NVFP4_EINVAL, "range %d [%lld, %lld) -> %lld: bounds must be multiples of 64 within [0, N]", i,
+                  (long long)r.begin, (long long)r.end, (long long)r.dst_col);
+    if (r.act != NVFP4_ACT_NONE && r.act != NVFP4_ACT_GELU_TANH)
+      return fail(NVFP4_EINVAL, "range %d: unknown activation %d", i, r.act);
+    if (r.dst == NVFP4_DST_BF16) {
+      any_bf16 = true;
+      if (r.dst_col + (r.end - r.begin) > ldy) return fail(NVFP4_EINVAL, "range %d overruns ldy", i);
+    } else if (r.dst == NVFP4_DST_NVFP4) {
+      any_fp4 = true;
+      if (r.dst_col + (r.end - r.begin) > k_next) return fail(NVFP4_EINVAL, "range %d overruns k_next", i);
+    } else {
+      return fail(NVFP4_EINVAL, "range %d: unknown destination %d", i, r.dst);
+    }
+    for (int j = 0; j < i; ++j)
+      if (ranges[j].begin < r.end && r.begin < ranges[j].end)
+        return fail(NVFP4_EINVAL, "ranges %d and %d overlap", j, i);
+  }
+  if (any_bf16) {
+    if (!y_bf16) return fail(NVFP4_EINVAL, "a BF16 range needs y_bf16");
+    if (ldy < 8 || ldy % 8 != 0) return fail(NVFP4_EINVAL, "ldy=%lld must be a positive multiple of 8", (long long)ldy);
+    if (!aligned16(y_bf16)) return fail(NVFP4_EALIGN, "y_bf16 must be 16-byte aligned");
+  }
+  if (any_fp4) {
+    if (!codes_next || !sf_next) return fail(NVFP4_EINVAL, "an NVFP4 range needs codes_next and sf_next");
+    if (k_next < 64 || k_next % 64 != 0 || k_next > INT32_MAX / 2)
+      return fail(NVFP4_EINVAL, "k_next=%lld must be a positive multiple of 64", (long long)k_next);
+    if (!scale_ok(g_next)) return fail(NVFP4_EINVAL, "g_next must be finite and in [2^-64, 2^64]");
+    if (!aligned16(codes_next) || !aligned16(sf_next))
+      return fail(NVFP4_EALIGN, "codes_next and sf_next must be 16-byte aligned");
+  }
+  GemmParams p;
+  CUtensorMap ta, tb, ty;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &ta, &tb, &dev);
+  if (st != NVFP4_OK) return st;
+  if (any_bf16) {
+    st = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, ldy, M, ldy * 2, 32, 32,
+                   CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  } else {
+    // never used for a store; a valid descriptor keeps the prefetch harmless
+    st = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, 16, 1, 16, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE, "dummy");
+  }
+  if (st != NVFP4_OK) return st;
+  p.n_ranges = n_ranges;
+  for (int i = 0; i < n_ranges; ++i) {
+    p.ranges[i].begin = static_cast<int32_t>(ranges[i].begin);
+    p.ranges[i].end = static_cast<int32_t>(ranges[i].end);
+    p.ranges[i].act = ranges[i].act;
+    p.ranges[i].dst = ranges[i].dst;
+    p.ranges[i].dst_col = static_cast<int32_t>(ranges[i].dst_col);
+  }
+  p.g_next = g_next;
+  p.codes_next = codes_next;
+  p.sf_next = sf_next;
+  p.k_next = static_cast<int32_t>(k_next);
+  cudaError_t e = launch_gemm(ta, tb, ty, p, true, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_quant launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_check_fault(void) {
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_fault_word, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read fault word");
+  if (v != 0u) {
+    const unsigned zero = 0u;
+    e = cudaMemcpyToSymbol(g_fault_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clear fault word");
+    return fail(NVFP4_ETIMEOUT, "a kernel gave up waiting on a barrier (fault bits 0x%x)", v);
+  }
+  return ok();
+}
+
+const char* nvfp4_last_error(void) { return t_last_error.c_str(); }
+
+}  // extern "C"

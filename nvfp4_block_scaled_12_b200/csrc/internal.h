@@ -1,0 +1,56 @@
+// Declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device.cuh"
+#include "nvfp4.h"
+
+namespace nvfp4 {
+
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  size_t max_smem_optin = 0;
+  unsigned* fault = nullptr;  // device address of the fault word
+};
+
+// One column range of the fused epilogue, as the kernel sees it.
+struct EpiRange {
+  int32_t begin, end, act, dst, dst_col;
+};
+
+struct GemmParams {
+  int32_t M, N, K;
+  int32_t tiles_m, tiles_n, num_tiles;
+  int32_t num_kt;   // k-tiles of 256 elements (last one may be partial)
+  int32_t k64;      // K / 64: MMA k-blocks in total, and scale atoms per 128-row block
+  int32_t sfb_row_blocks;  // ceil(N / 128)
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  float alpha;
+  const __nv_bfloat16* bias;  // nullable
+  unsigned* fault;
+  // fused epilogue (only read by the fused kernel)
+  int32_t n_ranges;
+  EpiRange ranges[NVFP4_MAX_RANGES];
+  float g_next;
+  uint8_t* codes_next;
+  uint8_t* sf_next;
+  int32_t k_next;
+};
+
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
+                            cudaStream_t stream, const DeviceInfo& dev);
+cudaError_t launch_calibrate(const void* x, int64_t n, float* out, cudaStream_t stream, const DeviceInfo& dev);
+cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out, cudaStream_t stream);
+
+// tmap_y describes the bf16 destination of the plain epilogue, or the bf16
+// destination of BF16 ranges for the fused one (may be unused).
+cudaError_t launch_gemm(const CUtensorMap& tmap_a, const CUtensorMap& tmap_b, const CUtensorMap& tmap_y,
+                        const GemmParams& p, bool fused, cudaStream_t stream, const DeviceInfo& dev);
+
+}  // namespace nvfp4

@@ -1,0 +1,104 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+function include/nvfp4.h declares, and rejects invalid arguments before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_12_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    for n in ("nvfp4_sf_bytes", "nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm",
+              "nvfp4_gemm_quant", "nvfp4_check_fault", "nvfp4_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(F.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_mirrors_every_entry_point():
+    for n in declared_functions():
+        assert callable(getattr(F, n, None)), n
+
+
+@pytest.mark.parametrize("rows,k,want", [(4608, 12288, 4608 * 768), (1, 64, 128 * 4), (129, 16, 256 * 4),
+                                         (0, 64, 0), (5, 8, 0), (5, 24, 0)])
+def test_sf_bytes(rows, k, want):
+    assert F.nvfp4_sf_bytes(rows, k) == want
+
+
+def _expect(status, fn, *args):
+    with pytest.raises(F.NVFP4Error) as e:
+        fn(*args)
+    assert e.value.status == status, str(e.value)
+    assert F.nvfp4_last_error()
+
+
+P = 1 << 20  # a 16-byte-aligned fake device address: never dereferenced
+
+
+def test_quantize_rejects_bad_arguments_on_the_host():
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, 0, 16, 64, 1.0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, 0, 64, 1.0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, 4, 48, 1.0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, 4, 64, float("nan"), P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, 4, 64, 0.0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, 4, 64, 2.0 ** 70, P, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_quantize, P + 2, 4, 64, 1.0, P, P, 0)
+
+
+def test_gemm_rejects_bad_arguments_on_the_host():
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, 0, 64, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, 16, 12, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, 16, 64, 96, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, 16, 64, 64, float("inf"), 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, 0, P, P, 16, 64, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_gemm, P, P, P + 8, P, 16, 64, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_gemm, P, P, P, P, 16, 64, 64, 1.0, P + 4, P, 0)
+
+
+def test_gemm_quant_rejects_bad_ranges_on_the_host():
+    R = F.ColRange
+    args = lambda rs: (P, P, P, P, 128, 256, 256, 1.0, 0, rs, P, 256, 0.1, P, P, 256, 0)  # noqa: E731
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 100, 0, 1, 0)]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 128, 0, 1, 0), R(64, 192, 0, 0, 0)]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 128, 7, 1, 0)]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 128, 0, 9, 0)]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 512, 0, 1, 0)]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 256, 0, 1, 64)]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([]))
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 64, 0, 1, 0)] * 9))
+
+
+def test_calibrate_and_swizzle_reject_bad_arguments_on_the_host():
+    _expect(F.NVFP4_EINVAL, F.nvfp4_calibrate, P, 12, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_calibrate, P + 1, 16, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_swizzle_sf, P, 4, 80, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_swizzle_sf, P, 4, 64, P + 4, 0)
+
+
+def test_valid_arguments_without_a_device_fail_loudly_not_silently():
+    # On this CPU-only host a valid call reaches the device check and must
+    # report an error: there is no CPU fallback.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(F.NVFP4Error) as e:
+        F.nvfp4_quantize(P, 4, 64, 1.0, P, P, 0)
+    assert e.value.status in (F.NVFP4_ECUDA, F.NVFP4_EARCH)
