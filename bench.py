@@ -313,6 +313,20 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
 
+    # the standalone activation-quantize workload, bf16 [4608, 12288]
+    xl = synth.quantize_input().to(device)
+    gl = F.global_scale(xl)
+    xlq = F.quantize(xl, gl)
+    ql_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    for a, b in ql_ev:
+        flush.zero_()
+        a.record(stream)
+        F.quantize(xl, gl, out=xlq, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    ql_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ql_ev[3:]), world, device)
+    F.nvfp4_check_fault()
+
     if rank == 0:
         hbm, bf16, src = peaks()
         fp4_peak = bf16 * FP4_PER_BF16
@@ -342,6 +356,10 @@ def run_ours(args):
                 "gemm": {"ms": gemm_ms, "tflops": gemm_tf, "frac_of_fp4_peak": gemm_tf / fp4_peak},
                 "quantize": {"ms": quant_ms, "gbs": quant_gbs, "frac_of_hbm": quant_gbs / hbm,
                              "bytes": M * K * QUANT_BYTES_PER_ELEM, "hbm_peak_gbs": hbm, "peak_source": src},
+                "quantize_4608x12288": {
+                    "ms": ql_ms, "gbs": xl.numel() * QUANT_BYTES_PER_ELEM / (ql_ms * 1e-3) / 1e9,
+                    "frac_of_hbm": xl.numel() * QUANT_BYTES_PER_ELEM / (ql_ms * 1e-3) / 1e9 / hbm,
+                    "note": "standalone quantize workload (Laplace, spikes, zero blocks), median of 17, L2 flushed"},
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},

@@ -4,21 +4,26 @@
 // epilogue and an optional fused epilogue that quantizes the result for the
 // next layer.
 //
-// Design (one persistent CTA per SM, 6 warps, warp-specialised):
+// Design (one persistent CTA per SM, 10 warps, warp-specialised):
 //   warp 0      TMA producer: 128x256 A tile, 192x256 B tile and their scale
 //               atoms into a 4-stage shared-memory ring (mbarrier expect-tx).
-//   warp 1      allocates TMEM; one thread copies each stage's scale atoms
-//               into TMEM (tcgen05.cp) and issues tcgen05.mma
-//               kind::mxf4nvf4 (M=128, N=192, K=64, one UE4M3 scale per 16
-//               elements) into a double-buffered fp32 accumulator in TMEM.
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma kind::mxf4nvf4
+//               (M=128, N=192, K=64, one UE4M3 scale per 16 elements) into a
+//               double-buffered fp32 accumulator in TMEM.
 //   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, alpha*acc + bias,
 //               bf16, swizzled staging in shared memory, TMA store; they
 //               drain accumulator i while the MMA fills accumulator i^1.
-// TMEM columns: [0,192) and [192,384) accumulators, [384,400) A scales,
-// [416,448) B scales.  Scale atoms in TMEM: atom column j of lane l holds the
-// 4 scales of row 32*j + l, so row i of a tile is read from column i/32; a
-// 192-wide B tile that starts at row 64 of a 128-row atom block skips 2
-// columns.
+//   warps 6-9   scale-factor movers: copy each stage's scale atoms from shared
+//               memory into a double-buffered TMEM slot with tcgen05.st, one
+//               warp per 32-lane TMEM quarter.  The MMA reads every scale row
+//               from all four quarters, so each quarter holds a full copy.
+//               Register-path stores run beside the tensor pipe; tcgen05.cp
+//               copies of the same data would serialize with the MMAs.
+// TMEM columns: [0,192) and [192,384) accumulators; [384,432) and [432,480)
+// scale slots, each 16 columns of A scales (4 per MMA k-block) then 32 of B
+// scales (8 per k-block).  Scale atom column j of lane l holds the 4 scales
+// of row 32*j + l, so row i of a tile is read from column i/32; a 192-wide B
+// tile that starts at row 64 of a 128-row atom block skips 2 columns.
 // Every barrier wait is bounded (see mbar_wait); a role that gives up sets
 // the CTA's abort flag and the device fault word, lets the copies it issued
 // land, and the CTA still frees its TMEM before exiting.
@@ -32,7 +37,7 @@ constexpr int kBM = 128;
 constexpr int kBN = 192;
 constexpr int kBKBytes = 128;  // 256 fp4 elements per row per stage
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kChunks = kBN / 32;
 
 constexpr uint32_t kABytes = kBM * kBKBytes;  // 16 KB
@@ -46,14 +51,15 @@ constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
 constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
 constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;  // 4 warps x 2 x 2 KB
 constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * 2048;
-constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1;
+constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1 + 2 + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = 384;
-constexpr uint32_t kSfbCol = 416;
-static_assert(2 * kBN <= kSfaCol && kSfbCol + 32 <= kTmemCols, "TMEM layout");
+constexpr uint32_t kSfCol = 384;       // first scale slot
+constexpr uint32_t kSfSlotCols = 48;   // 16 A-scale + 32 B-scale columns per k-tile
+constexpr uint32_t kSfbOff = 16;       // B scales inside a slot
+static_assert(2 * kBN <= kSfCol && kSfCol + 2 * kSfSlotCols <= kTmemCols, "TMEM layout");
 static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
 
 __device__ __forceinline__ float gelu_tanh_f32(float v) {
@@ -96,6 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = bars + 2 * kStages + 2;
   uint64_t* drain = bars + 2 * kStages + 4;
+  uint64_t* sf_full = bars + 2 * kStages + 5;
+  uint64_t* sf_empty = bars + 2 * kStages + 7;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -112,6 +120,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[a], 4);
     }
     mbar_init(drain, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sf_full[t], 4);
+      mbar_init(&sf_empty[t], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -180,11 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
       int stage = 0;
       uint32_t phase = 0;
+      int slot = 0;
+      uint32_t slot_phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = blockIdx.x; tile < p.num_tiles && fault == 0u; tile += gridDim.x) {
         const int n0 = (tile / p.tiles_m) * kBN;
-        const bool has_rb1 = (n0 >> 7) + 1 < p.sfb_row_blocks;
         const uint32_t sfb_shift = (n0 & 127) ? 2u : 0u;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
           fault = kFaultMmaWait;
@@ -193,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag) || !mbar_wait(&sf_full[slot], slot_phase, abort_flag)) {
             fault = kFaultMmaWait;
             break;
           }
@@ -201,24 +214,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nkb = min(4, p.k64 - kt * 4);
           const uint32_t sa = smem_u32(smem + kOffA + stage * kABytes);
           const uint32_t sb = smem_u32(smem + kOffB + stage * kBBytes);
-          const uint32_t ssfa = smem_u32(smem + kOffSfa + stage * kSfaBytes);
-          const uint32_t ssfb = smem_u32(smem + kOffSfb + stage * kSfbBytes);
-          for (int kb = 0; kb < nkb; ++kb) {
-            tc_cp_32x128b_warpx4(tmem_base + kSfaCol + kb * 4, sdesc_sf_atom(ssfa + kb * 512));
-            tc_cp_32x128b_warpx4(tmem_base + kSfbCol + kb * 8, sdesc_sf_atom(ssfb + kb * 512));
-            if (has_rb1)
-              tc_cp_32x128b_warpx4(tmem_base + kSfbCol + kb * 8 + 4, sdesc_sf_atom(ssfb + 4 * 512 + kb * 512));
-          }
+          const uint32_t sf = tmem_base + kSfCol + static_cast<uint32_t>(slot) * kSfSlotCols;
           for (int kb = 0; kb < nkb; ++kb) {
             tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sa + kb * 32), sdesc_kmajor_sw128(sb + kb * 32), idesc,
-                        tmem_base + kSfaCol + kb * 4, tmem_base + kSfbCol + kb * 8 + sfb_shift,
-                        (kt | kb) != 0 ? 1u : 0u);
+                        sf + kb * 4, sf + kSfbOff + kb * 8 + sfb_shift, (kt | kb) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          tc_commit(&empty[stage]);    // frees the smem stage once these MMAs have read it
+          tc_commit(&sf_empty[slot]);  // and the scale slot
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
+          slot ^= 1;
+          if (slot == 0) slot_phase ^= 1u;
         }
         if (fault != 0u) break;
         tc_commit(&acc_full[acc]);  // accumulator ready for the epilogue
@@ -231,6 +239,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(drain, 0u, nullptr)) fault |= kFaultDrainWait;
     }
     __syncwarp();
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ scale movers
+    const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter of this warp
+    int stage = 0;
+    uint32_t phase = 0;
+    int slot = 0;
+    uint32_t slot_phase = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles && fault == 0u; tile += gridDim.x) {
+      for (int kt = 0; kt < p.num_kt; ++kt) {
+        const bool got = mbar_wait(&full[stage], phase, abort_flag) &&
+                         mbar_wait(&sf_empty[slot], slot_phase ^ 1u, abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got)) {
+          fault = kFaultMmaWait;
+          break;
+        }
+        tc_fence_after();
+        const int nkb = min(4, p.k64 - kt * 4);
+        const uint8_t* ssfa = smem + kOffSfa + stage * kSfaBytes + lane * 16;
+        const uint8_t* ssfb = smem + kOffSfb + stage * kSfbBytes + lane * 16;
+        const uint32_t t = tmem_base + ((q * 32u) << 16) + kSfCol + static_cast<uint32_t>(slot) * kSfSlotCols;
+        for (int kb = 0; kb < nkb; ++kb) {
+          const uint4 a = *reinterpret_cast<const uint4*>(ssfa + kb * 512);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 4 * 512 + kb * 512);
+          tmem_st_32x32b_x4(t + kb * 4, a);
+          tmem_st_32x32b_x8(t + kSfbOff + kb * 8, b0, b1);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[slot]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        slot ^= 1;
+        if (slot == 0) slot_phase ^= 1u;
+      }
+    }
+    if (fault != 0u) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
