@@ -11,8 +11,6 @@
 
 namespace nvfp4 {
 
-int gemm_tile_n();
-
 namespace {
 
 // Fault word: kernels OR a code in here when a barrier wait times out.
@@ -97,30 +95,57 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Row-major tensor of `rank` dims (innermost first) with byte strides of
+// dims 1.. in `strides`.
+nvfp4_status make_tmap_nd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank, const uint64_t* dims,
+                          const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(NVFP4_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+  const CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, bx, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NVFP4_ECUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
+  return NVFP4_OK;
+}
+
 // 2-D row-major tensor [outer, inner] with rows `row_bytes` apart.
 nvfp4_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw,
                        const char* what) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return fail(NVFP4_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(NVFP4_ECUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
-  return NVFP4_OK;
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {row_bytes};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return make_tmap_nd(m, dt, base, 2, dims, strides, box, sw, what);
+}
+
+// Swizzled scale buffer of a [rows, k] tensor seen as [row blocks][k/64
+// atoms][128 x u32]; the box covers 4 atoms (one 256-wide k-tile) of
+// `box_blocks` row blocks.  Out-of-range atoms and blocks read as zero.
+nvfp4_status make_sf_tmap(CUtensorMap* m, const void* sf, int64_t rows, int64_t k, uint32_t box_blocks,
+                          const char* what) {
+  const uint64_t dims[3] = {128, static_cast<uint64_t>(k / 64), static_cast<uint64_t>((rows + 127) / 128)};
+  const uint64_t strides[2] = {512, static_cast<uint64_t>(k / 64) * 512};
+  const uint32_t box[3] = {128, 4, box_blocks};
+  return make_tmap_nd(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, sf, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      what);
 }
 
 bool finite_f(float v) { return isfinite(v) != 0; }
 
 bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
 
-// Checks shared by the two GEMM entry points; fills the operand part of p.
+// Checks shared by the two GEMM entry points; fills the operand part of p
+// and the operand tensor maps.
 nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
-                         int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, CUtensorMap* ta,
-                         CUtensorMap* tb, const DeviceInfo** dev) {
+                         int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, GemmTensorMaps* maps,
+                         GemmConfig* cfg, const DeviceInfo** dev) {
   if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
   if (M < 1 || M > INT32_MAX / 2) return fail(NVFP4_EINVAL, "M=%lld out of range", (long long)M);
   if (N < 8 || N % 8 != 0 || N > INT32_MAX / 2)
@@ -133,29 +158,36 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   nvfp4_status st = current_device(dev);
   if (st != NVFP4_OK) return st;
 
-  const int bn = gemm_tile_n();
+  *cfg = gemm_config(M, N);
+  const int bn = cfg->tile_n;
+  const int cg = cfg->cta_group;
   *p = GemmParams{};
   p->M = static_cast<int32_t>(M);
   p->N = static_cast<int32_t>(N);
   p->K = static_cast<int32_t>(K);
-  p->tiles_m = static_cast<int32_t>((M + 127) / 128);
+  p->tiles_m = static_cast<int32_t>((M + 128 * cg - 1) / (128 * cg));
   p->tiles_n = static_cast<int32_t>((N + bn - 1) / bn);
   const int64_t tiles = static_cast<int64_t>(p->tiles_m) * p->tiles_n;
   if (tiles > INT32_MAX) return fail(NVFP4_EINVAL, "problem too large");
   p->num_tiles = static_cast<int32_t>(tiles);
   p->num_kt = static_cast<int32_t>((K + 255) / 256);
   p->k64 = static_cast<int32_t>(K / 64);
-  p->sfb_row_blocks = static_cast<int32_t>((N + 127) / 128);
-  p->sfa = sfa;
-  p->sfb = sfb;
   p->alpha = alpha;
   p->bias = static_cast<const __nv_bfloat16*>(bias);
   p->fault = (*dev)->fault;
 
-  st = make_tmap(ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+  st = make_tmap(&maps->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+                 "A");
   if (st != NVFP4_OK) return st;
-  st = make_tmap(tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, bn, CU_TENSOR_MAP_SWIZZLE_128B, "B");
-  return st;
+  st = make_tmap(&maps->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, bn / cg,
+                 CU_TENSOR_MAP_SWIZZLE_128B, "B");
+  if (st != NVFP4_OK) return st;
+  st = make_sf_tmap(&maps->sfa, sfa, M, K, 1, "A scales");
+  if (st != NVFP4_OK) return st;
+  // 128-row scale blocks one B tile can touch: a width that is not a
+  // multiple of 128 may start in the middle of a block
+  const uint32_t sfb_blocks = static_cast<uint32_t>(bn % 128 == 0 ? bn / 128 : bn / 128 + 1);
+  return make_sf_tmap(&maps->sfb, sfb, N, K, sfb_blocks, "B scales");
 }
 
 }  // namespace
@@ -220,13 +252,14 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, 
   if (!y) return fail(NVFP4_EINVAL, "null output pointer");
   if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
   GemmParams p;
-  CUtensorMap ta, tb, ty;
+  GemmTensorMaps maps;
+  GemmConfig cg;
   const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &ta, &tb, &dev);
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev);
   if (st != NVFP4_OK) return st;
-  st = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_gemm(ta, tb, ty, p, false, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_gemm(maps, p, cg, false, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return ok();
 }
@@ -273,16 +306,18 @@ nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_
       return fail(NVFP4_EALIGN, "codes_next and sf_next must be 16-byte aligned");
   }
   GemmParams p;
-  CUtensorMap ta, tb, ty;
+  GemmTensorMaps maps;
+  GemmConfig cg;
   const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &ta, &tb, &dev);
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev);
   if (st != NVFP4_OK) return st;
   if (any_bf16) {
-    st = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, ldy, M, ldy * 2, 32, 32,
+    st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, ldy, M, ldy * 2, 32, 32,
                    CU_TENSOR_MAP_SWIZZLE_64B, "Y");
   } else {
     // never used for a store; a valid descriptor keeps the prefetch harmless
-    st = make_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, 16, 1, 16, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE, "dummy");
+    st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, 16, 1, 16, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   "dummy");
   }
   if (st != NVFP4_OK) return st;
   p.n_ranges = n_ranges;
@@ -297,7 +332,7 @@ nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_
   p.codes_next = codes_next;
   p.sf_next = sf_next;
   p.k_next = static_cast<int32_t>(k_next);
-  cudaError_t e = launch_gemm(ta, tb, ty, p, true, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_gemm(maps, p, cg, true, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_quant launch");
   return ok();
 }

@@ -4,63 +4,83 @@
 // epilogue and an optional fused epilogue that quantizes the result for the
 // next layer.
 //
-// Design (one persistent CTA per SM, 10 warps, warp-specialised):
-//   warp 0      TMA producer: 128x256 A tile, 192x256 B tile and their scale
-//               atoms into a 4-stage shared-memory ring (mbarrier expect-tx).
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma kind::mxf4nvf4
-//               (M=128, N=192, K=64, one UE4M3 scale per 16 elements) into a
-//               double-buffered fp32 accumulator in TMEM.
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, alpha*acc + bias,
-//               bf16, swizzled staging in shared memory, TMA store; they
-//               drain accumulator i while the MMA fills accumulator i^1.
-//   warps 6-9   scale-factor movers: copy each stage's scale atoms from shared
-//               memory into a double-buffered TMEM slot with tcgen05.st, one
-//               warp per 32-lane TMEM quarter.  The MMA reads every scale row
-//               from all four quarters, so each quarter holds a full copy.
-//               Register-path stores run beside the tensor pipe; tcgen05.cp
-//               copies of the same data would serialize with the MMAs.
+// One persistent kernel, templated on the CTA-group size kCG:
+//   kCG = 2  a CTA pair (cluster of 2) owns a 256 x 192 output tile: each
+//            CTA loads its 128 rows of A and its 96 rows of B, and the pair
+//            leader issues tcgen05.mma.cta_group::2 (M=256, N=192, K=64), so
+//            every B byte crosses L2 once per pair.  Used for M > 128.
+//   kCG = 1  one CTA owns a 128 x 192 tile (small M).
+// Warps (10 per CTA):
+//   0     TMA producer: A/B tiles (128-byte rows, 128-byte swizzle) and the
+//         scale atoms (3-D boxes, zero-filled past K and past the last row
+//         block) into a shared-memory ring.
+//   1     allocates TMEM; in the leader one thread issues the MMAs into a
+//         double-buffered fp32 accumulator.
+//   2-5   epilogue: tcgen05.ld 32 columns at a time, alpha*acc + bias, bf16,
+//         swizzled staging in shared memory, TMA store (or the fused
+//         quantize); drains accumulator i while the MMA fills i^1.
+//   6-9   scale movers: copy each stage's scale atoms from shared memory into
+//         a double-buffered TMEM slot with tcgen05.st, one warp per 32-lane
+//         TMEM quarter.  The MMA reads every scale row from all four quarters,
+//         so each quarter holds a full copy.  Register-path stores run beside
+//         the tensor pipe, where tcgen05.cp copies of the same (replicated)
+//         data would serialize with the MMAs.
 // TMEM columns: [0,192) and [192,384) accumulators; [384,432) and [432,480)
 // scale slots, each 16 columns of A scales (4 per MMA k-block) then 32 of B
-// scales (8 per k-block).  Scale atom column j of lane l holds the 4 scales
-// of row 32*j + l, so row i of a tile is read from column i/32; a 192-wide B
-// tile that starts at row 64 of a 128-row atom block skips 2 columns.
+// scales (8 per k-block, covering two 128-row atom blocks).  Scale column j
+// of lane l holds the 4 scales of row 32*j + l, so row i of a tile is read
+// from column i/32; a 192-wide B tile that starts at row 64 of a 128-row atom
+// block skips 2 columns.
 // Every barrier wait is bounded (see mbar_wait); a role that gives up sets
 // the CTA's abort flag and the device fault word, lets the copies it issued
-// land, and the CTA still frees its TMEM before exiting.
+// land, and the CTA still reaches the final barrier and frees its TMEM.
 #include "internal.h"
 
 namespace nvfp4 {
 
 namespace {
 
-constexpr int kBM = 128;
-constexpr int kBN = 192;
-constexpr int kBKBytes = 128;  // 256 fp4 elements per row per stage
-constexpr int kStages = 4;
-constexpr int kThreads = 320;
-constexpr int kChunks = kBN / 32;
-
-constexpr uint32_t kABytes = kBM * kBKBytes;  // 16 KB
-constexpr uint32_t kBBytes = kBN * kBKBytes;  // 24 KB
+constexpr int kBKBytes = 128;   // 256 fp4 elements per row per stage
+constexpr uint32_t kABytes = 128 * kBKBytes;  // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t kSfaBytes = 4 * 512;       // 4 k-blocks x one 128-row atom
-constexpr uint32_t kSfbBytes = 2 * 4 * 512;   // two 128-row atom blocks x 4 k-blocks
-
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
-constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
-constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;  // 4 warps x 2 x 2 KB
-constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * 2048;
-constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1 + 2 + 2;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfCol = 384;       // first scale slot
-constexpr uint32_t kSfSlotCols = 48;   // 16 A-scale + 32 B-scale columns per k-tile
-constexpr uint32_t kSfbOff = 16;       // B scales inside a slot
-static_assert(2 * kBN <= kSfCol && kSfCol + 2 * kSfSlotCols <= kTmemCols, "TMEM layout");
-static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
+
+// kCG: CTAs per tile; kBN: tile width; kAcc: accumulator buffers in TMEM.
+template <int kCG, int kBN, int kAcc>
+struct Cfg {
+  static constexpr int kBNc = kBN / kCG;  // B rows per CTA
+  static constexpr uint32_t kBBytes = kBNc * kBKBytes;
+  static constexpr int kChunks = kBN / 32;
+  // 128-row scale blocks a B tile can touch (a 192-wide tile may start mid-block)
+  static constexpr int kSfbBlocks = kBN % 128 == 0 ? kBN / 128 : kBN / 128 + 1;
+  static constexpr uint32_t kSfbBytes = kSfbBlocks * 4 * 512;
+  // TMEM: accumulators, then a ring of per-k-tile scale slots
+  static constexpr uint32_t kSfCol = kAcc * kBN;
+  static constexpr uint32_t kSfbOff = 16;  // 16 A-scale columns, then 4 per B block per k-block
+  static constexpr uint32_t kSfSlotCols = 16 + 16 * kSfbBlocks;
+  static constexpr int kSfSlots = (kTmemCols - kSfCol) / kSfSlotCols > 8 ? 8 : (kTmemCols - kSfCol) / kSfSlotCols;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStagesFit = (224 * 1024 - 4 * 2 * 2048) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
+  static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
+  static constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
+  static constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;  // 4 warps x 2 x 2 KB
+  static constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * 2048;
+  // full, empty, sfin per stage; acc_full, acc_empty per accumulator;
+  // sf_full, sf_empty per scale slot; drain
+  static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAcc + 2 * kSfSlots + 1;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t kFullTx = kCG * (kABytes + kBBytes);  // A/B bytes of the whole group
+  static_assert(kBN % 32 == 0 && kBN / kCG % 8 == 0, "tile width");
+  static_assert(kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
+  static_assert(kSfSlots >= 2, "TMEM budget");
+  static_assert(kStages >= 3, "pipeline depth");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 __device__ __forceinline__ float gelu_tanh_f32(float v) {
   const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);
@@ -90,90 +110,119 @@ __device__ __forceinline__ void store_chunk_bf16(const CUtensorMap* tmap, uint8_
   }
 }
 
-template <bool kFused>
+template <int kCG, int kBN, int kAcc, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ GemmParams p) {
+  using C = Cfg<kCG, kBN, kAcc>;
+  constexpr int S = C::kStages;
+  constexpr int R = C::kSfSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* acc_full = bars + 2 * kStages;
-  uint64_t* acc_empty = bars + 2 * kStages + 2;
-  uint64_t* drain = bars + 2 * kStages + 4;
-  uint64_t* sf_full = bars + 2 * kStages + 5;
-  uint64_t* sf_empty = bars + 2 * kStages + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;            // leader: A/B of the whole group landed
+  uint64_t* empty = bars + S;       // this CTA's stage may be refilled
+  uint64_t* sfin = bars + 2 * S;    // this CTA's scale atoms landed
+  uint64_t* acc_full = bars + 3 * S;
+  uint64_t* acc_empty = acc_full + kAcc;   // leader
+  uint64_t* sf_full = acc_empty + kAcc;    // leader
+  uint64_t* sf_empty = sf_full + R;
+  uint64_t* drain = sf_empty + R;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kCG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x / kCG;
+  const int num_clusters = gridDim.x / kCG;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfin[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kAcc; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 4 * kCG);
+    }
+    for (int r = 0; r < R; ++r) {
+      mbar_init(&sf_full[r], 4 * kCG);
+      mbar_init(&sf_empty[r], 1);
     }
     mbar_init(drain, 1);
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&sf_full[t], 4);
-      mbar_init(&sf_empty[t], 1);
-    }
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_sfa);
+    prefetch_tmap(&tmap_sfb);
     prefetch_tmap(&tmap_y);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<kCG>(tmem_slot, kTmemCols);
+    tmem_relinquish<kCG>();
   }
   tc_fence_before();
   __syncthreads();
+  if (kCG == 2) cluster_sync();  // the peer's barriers are initialised before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   unsigned fault = 0u;
+
+  // arrive on a barrier that lives in the group leader
+  auto arrive_leader = [&](uint64_t* bar) {
+    if (kCG == 2 && !leader)
+      mbar_arrive_cluster(peer_smem(smem_u32(bar), 0));
+    else
+      mbar_arrive(bar);
+  };
+  // commit to a barrier in every CTA of the group
+  auto commit_group = [&](uint64_t* bar) {
+    if (kCG == 2)
+      tc_commit_pair(bar, 0x3);
+    else
+      tc_commit(bar);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int last_phase[kStages];
+      int last_phase[S];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
-      for (int tile = blockIdx.x; tile < p.num_tiles && fault == 0u; tile += gridDim.x) {
+      for (int s = 0; s < S; ++s) last_phase[s] = -1;
+      for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
         const int tm = tile % p.tiles_m;
         const int n0 = (tile / p.tiles_m) * kBN;
-        const int rb0 = n0 >> 7;
-        const bool has_rb1 = rb0 + 1 < p.sfb_row_blocks;
+        const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
         for (int kt = 0; kt < p.num_kt; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             fault = kFaultProducerWait;
             break;
           }
-          const int nkb = min(4, p.k64 - kt * 4);
-          const uint32_t sf_bytes = static_cast<uint32_t>(nkb) * 512u;
-          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes + sf_bytes * (has_rb1 ? 3u : 2u));
-          tma_load_2d(smem + kOffA + stage * kABytes, &tmap_a, &full[stage], kt * kBKBytes, tm * kBM);
-          tma_load_2d(smem + kOffB + stage * kBBytes, &tmap_b, &full[stage], kt * kBKBytes, n0);
-          bulk_load(smem + kOffSfa + stage * kSfaBytes,
-                    p.sfa + (static_cast<size_t>(tm) * p.k64 + kt * 4) * 512, sf_bytes, &full[stage]);
-          bulk_load(smem + kOffSfb + stage * kSfbBytes,
-                    p.sfb + (static_cast<size_t>(rb0) * p.k64 + kt * 4) * 512, sf_bytes, &full[stage]);
-          if (has_rb1)
-            bulk_load(smem + kOffSfb + stage * kSfbBytes + 4 * 512,
-                      p.sfb + (static_cast<size_t>(rb0 + 1) * p.k64 + kt * 4) * 512, sf_bytes, &full[stage]);
+          if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
+          mbar_arrive_expect_tx(&sfin[stage], kSfaBytes + C::kSfbBytes);
+          uint8_t* sa = smem + C::kOffA + stage * kABytes;
+          uint8_t* sb = smem + C::kOffB + stage * C::kBBytes;
+          if (kCG == 2) {
+            const uint32_t fb = peer_smem(smem_u32(&full[stage]), 0);
+            tma_load_2d_pair(sa, &tmap_a, fb, kt * kBKBytes, row_block * 128);
+            tma_load_2d_pair(sb, &tmap_b, fb, kt * kBKBytes, n0 + static_cast<int>(rank) * C::kBNc);
+          } else {
+            tma_load_2d(sa, &tmap_a, &full[stage], kt * kBKBytes, row_block * 128);
+            tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
+          }
+          tma_load_3d(smem + C::kOffSfa + stage * kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * 4, row_block);
+          tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * 4, n0 >> 7);
           last_phase[stage] = static_cast<int>(phase);
-          if (++stage == kStages) {
+          if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
@@ -182,21 +231,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (fault != 0u) {
         *abort_flag = 1;
         // let every copy already issued land before shared memory goes away
-        for (int s = 0; s < kStages; ++s)
-          if (last_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(last_phase[s]), nullptr);
+        for (int s = 0; s < S; ++s) {
+          if (last_phase[s] < 0) continue;
+          mbar_wait(&sfin[s], static_cast<uint32_t>(last_phase[s]), nullptr);
+          if (leader) mbar_wait(&full[s], static_cast<uint32_t>(last_phase[s]), nullptr);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
+    // ------------------------------------------------------------ MMA issuer (group leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_nvf4(128 * kCG, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int slot = 0;
       uint32_t slot_phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < p.num_tiles && fault == 0u; tile += gridDim.x) {
+      for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
         const int n0 = (tile / p.tiles_m) * kBN;
         const uint32_t sfb_shift = (n0 & 127) ? 2u : 0u;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -206,36 +258,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag) || !mbar_wait(&sf_full[slot], slot_phase, abort_flag)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag) ||
+              !mbar_wait(&sf_full[slot], slot_phase, abort_flag)) {
             fault = kFaultMmaWait;
             break;
           }
           tc_fence_after();
           const int nkb = min(4, p.k64 - kt * 4);
-          const uint32_t sa = smem_u32(smem + kOffA + stage * kABytes);
-          const uint32_t sb = smem_u32(smem + kOffB + stage * kBBytes);
-          const uint32_t sf = tmem_base + kSfCol + static_cast<uint32_t>(slot) * kSfSlotCols;
+          const uint32_t sa = smem_u32(smem + C::kOffA + stage * kABytes);
+          const uint32_t sb = smem_u32(smem + C::kOffB + stage * C::kBBytes);
+          const uint32_t sf = tmem_base + C::kSfCol + static_cast<uint32_t>(slot) * C::kSfSlotCols;
           for (int kb = 0; kb < nkb; ++kb) {
-            tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(sa + kb * 32), sdesc_kmajor_sw128(sb + kb * 32), idesc,
-                        sf + kb * 4, sf + kSfbOff + kb * 8 + sfb_shift, (kt | kb) != 0 ? 1u : 0u);
+            const uint64_t ad = sdesc_kmajor_sw128(sa + kb * 32), bd = sdesc_kmajor_sw128(sb + kb * 32);
+            const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
+            const uint32_t sfb = sf + C::kSfbOff + kb * 4 * C::kSfbBlocks + sfb_shift;
+            if (kCG == 2)
+              tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, sf + kb * 4, sfb, accum);
+            else
+              tc_mma_nvf4(d_tmem, ad, bd, idesc, sf + kb * 4, sfb, accum);
           }
-          tc_commit(&empty[stage]);    // frees the smem stage once these MMAs have read it
-          tc_commit(&sf_empty[slot]);  // and the scale slot
-          if (++stage == kStages) {
+          commit_group(&empty[stage]);    // frees the smem stages once these MMAs have read them
+          commit_group(&sf_empty[slot]);  // and the scale slots
+          if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
-          slot ^= 1;
-          if (slot == 0) slot_phase ^= 1u;
+          if (++slot == R) {
+            slot = 0;
+            slot_phase ^= 1u;
+          }
         }
         if (fault != 0u) break;
-        tc_commit(&acc_full[acc]);  // accumulator ready for the epilogue
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        commit_group(&acc_full[acc]);  // accumulators ready for both epilogues
+        if (++acc == kAcc) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (fault != 0u) *abort_flag = 1;
       // every tcgen05 op issued must complete before TMEM is released
-      tc_commit(drain);
+      if (kCG == 2)
+        tc_commit_pair_local(drain);
+      else
+        tc_commit(drain);
       if (!mbar_wait(drain, 0u, nullptr)) fault |= kFaultDrainWait;
     }
     __syncwarp();
@@ -246,9 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     int slot = 0;
     uint32_t slot_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles && fault == 0u; tile += gridDim.x) {
+    for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
       for (int kt = 0; kt < p.num_kt; ++kt) {
-        const bool got = mbar_wait(&full[stage], phase, abort_flag) &&
+        const bool got = mbar_wait(&sfin[stage], phase, abort_flag) &&
                          mbar_wait(&sf_empty[slot], slot_phase ^ 1u, abort_flag);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
@@ -257,37 +322,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const int nkb = min(4, p.k64 - kt * 4);
-        const uint8_t* ssfa = smem + kOffSfa + stage * kSfaBytes + lane * 16;
-        const uint8_t* ssfb = smem + kOffSfb + stage * kSfbBytes + lane * 16;
-        const uint32_t t = tmem_base + ((q * 32u) << 16) + kSfCol + static_cast<uint32_t>(slot) * kSfSlotCols;
+        const uint8_t* ssfa = smem + C::kOffSfa + stage * kSfaBytes + lane * 16;
+        const uint8_t* ssfb = smem + C::kOffSfb + stage * C::kSfbBytes + lane * 16;
+        const uint32_t t =
+            tmem_base + ((q * 32u) << 16) + C::kSfCol + static_cast<uint32_t>(slot) * C::kSfSlotCols;
         for (int kb = 0; kb < nkb; ++kb) {
           const uint4 a = *reinterpret_cast<const uint4*>(ssfa + kb * 512);
-          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512);
-          const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 4 * 512 + kb * 512);
           tmem_st_32x32b_x4(t + kb * 4, a);
-          tmem_st_32x32b_x8(t + kSfbOff + kb * 8, b0, b1);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512);
+          if (C::kSfbBlocks == 2) {
+            const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 4 * 512 + kb * 512);
+            tmem_st_32x32b_x8(t + C::kSfbOff + kb * 8, b0, b1);
+          } else {
+            tmem_st_32x32b_x4(t + C::kSfbOff + kb * 4, b0);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_full[slot]);
-        if (++stage == kStages) {
+        if (lane == 0) arrive_leader(&sf_full[slot]);
+        if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
-        slot ^= 1;
-        if (slot == 0) slot_phase ^= 1u;
+        if (++slot == R) {
+          slot = 0;
+          slot_phase ^= 1u;
+        }
       }
     }
     if (fault != 0u) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint8_t* stage_buf = smem + kOffEpi + (warp - 2) * 4096;
+    uint8_t* stage_buf = smem + C::kOffEpi + (warp - 2) * 4096;
     int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    const int m_padded = (p.M + 127) & ~127;  // rows of the next layer's scale buffer
+    for (int tile = cluster; tile < p.num_tiles; tile += num_clusters) {
       const int tm = tile % p.tiles_m;
       const int n0 = (tile / p.tiles_m) * kBN;
       const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
@@ -297,20 +370,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row_base = tm * kBM + q * 32;
+      const int row_base = (tm * kCG + static_cast<int>(rank)) * 128 + q * 32;
       const int row = row_base + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
       uint32_t sf_word = 0u;
 #pragma unroll 1
-      for (int c = 0; c < kChunks; ++c) {
+      for (int c = 0; c < C::kChunks; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
         tmem_ld_wait(r);
-        if (c == kChunks - 1) {
-          // accumulator fully read: hand it back to the MMA warp
+        if (c == C::kChunks - 1) {
+          // accumulator fully read: hand it back to the MMA issuer
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (lane == 0) arrive_leader(&acc_empty[acc]);
         }
         const int n = n0 + c * 32;
         if (n >= p.N) continue;
@@ -376,13 +449,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           sf_word |= (s0 | (s1 << 8)) << (8 * (csf & 3));
           if ((csf & 3) == 2) {  // the 64-column group is complete
             const uint32_t word = row < p.M ? sf_word : 0u;  // padding rows of the scale buffer are zero
-            *reinterpret_cast<uint32_t*>(p.sf_next + sf_offset(row, csf & ~3, p.k_next >> 6)) = word;
+            if (row < m_padded)
+              *reinterpret_cast<uint32_t*>(p.sf_next + sf_offset(row, csf & ~3, p.k_next >> 6)) = word;
             sf_word = 0u;
           }
         }
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == kAcc) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     if (lane == 0) bulk_wait<0>();
     if (fault != 0u) *abort_flag = 1;
@@ -391,25 +467,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (fault != 0u && lane == 0 && p.fault != nullptr) atomicOr(p.fault, fault);
   tc_fence_before();
   __syncthreads();
+  if (kCG == 2) cluster_sync();  // the peer no longer reads this CTA's smem or signals its barriers
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc<kCG>(tmem_base, kTmemCols);
   }
+}
+
+template <int kCG, int kBN, int kAcc, bool kFused>
+cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t stream, const DeviceInfo& dev) {
+  using C = Cfg<kCG, kBN, kAcc>;
+  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kCG == 2 ? 1 : 0;
+  // A persistent grid must be co-resident: as many CTA groups as fit at once.
+  static int max_groups = 0;  // per template instance; one device family
+  if (max_groups == 0) {
+    int n = dev.num_sms / kCG;
+    if (kCG == 2) {
+      cfg.gridDim = dim3(static_cast<unsigned>(2 * n), 1, 1);
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) == cudaSuccess && clusters > 0 && clusters < n)
+        n = clusters;
+    }
+    max_groups = n;
+  }
+  const int groups = p.num_tiles < max_groups ? p.num_tiles : max_groups;
+  cfg.gridDim = dim3(static_cast<unsigned>(groups * kCG), 1, 1);
+  err = cudaLaunchKernelEx(&cfg, kernel, m.a, m.b, m.sfa, m.sfb, m.y, p);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(const CUtensorMap& tmap_a, const CUtensorMap& tmap_b, const CUtensorMap& tmap_y,
-                        const GemmParams& p, bool fused, cudaStream_t stream, const DeviceInfo& dev) {
-  auto kernel = fused ? gemm_nvf4_kernel<true> : gemm_nvf4_kernel<false>;
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (err != cudaSuccess) return err;
-  const int grid = p.num_tiles < dev.num_sms ? p.num_tiles : dev.num_sms;
-  kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap_a, tmap_b, tmap_y, p);
-  return cudaGetLastError();
+GemmConfig gemm_config(int64_t M, int64_t N) {
+  (void)N;
+  if (M > 128) return GemmConfig{2, 192, 2};
+  return GemmConfig{1, 192, 2};
 }
 
-int gemm_tile_n() { return kBN; }
+cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused,
+                        cudaStream_t stream, const DeviceInfo& dev) {
+#define NVFP4_GEMM_CASE(CG, BN, ACC)                                                                          \
+  if (c.cta_group == CG && c.tile_n == BN && c.acc_bufs == ACC)                                             \
+    return fused ? launch<CG, BN, ACC, true>(m, p, stream, dev) : launch<CG, BN, ACC, false>(m, p, stream, dev);
+  NVFP4_GEMM_CASE(2, 192, 2)
+  NVFP4_GEMM_CASE(1, 192, 2)
+  NVFP4_GEMM_CASE(2, 128, 2)
+  NVFP4_GEMM_CASE(1, 128, 2)
+  NVFP4_GEMM_CASE(2, 256, 1)
+#undef NVFP4_GEMM_CASE
+  return cudaErrorInvalidConfiguration;
+}
 
 }  // namespace nvfp4

@@ -25,12 +25,9 @@ struct EpiRange {
 
 struct GemmParams {
   int32_t M, N, K;
-  int32_t tiles_m, tiles_n, num_tiles;
-  int32_t num_kt;   // k-tiles of 256 elements (last one may be partial)
-  int32_t k64;      // K / 64: MMA k-blocks in total, and scale atoms per 128-row block
-  int32_t sfb_row_blocks;  // ceil(N / 128)
-  const uint8_t* sfa;
-  const uint8_t* sfb;
+  int32_t tiles_m, tiles_n, num_tiles;  // tiles_m counts (128 * CTA-group)-row tiles
+  int32_t num_kt;  // k-tiles of 256 elements (last one may be partial)
+  int32_t k64;     // K / 64: MMA k-blocks in total, and scale atoms per 128-row block
   float alpha;
   const __nv_bfloat16* bias;  // nullable
   unsigned* fault;
@@ -43,14 +40,26 @@ struct GemmParams {
   int32_t k_next;
 };
 
+// TMA descriptors of one GEMM launch.
+struct GemmTensorMaps {
+  CUtensorMap a, b;      // codes, [rows, K/2] uint8, 128-byte swizzle
+  CUtensorMap sfa, sfb;  // swizzled scales as [row blocks][K/64 atoms][128 x u32]
+  CUtensorMap y;         // bf16 destination of the plain or BF16-range epilogue
+};
+
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
                             cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_calibrate(const void* x, int64_t n, float* out, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out, cudaStream_t stream);
 
-// tmap_y describes the bf16 destination of the plain epilogue, or the bf16
-// destination of BF16 ranges for the fused one (may be unused).
-cudaError_t launch_gemm(const CUtensorMap& tmap_a, const CUtensorMap& tmap_b, const CUtensorMap& tmap_y,
-                        const GemmParams& p, bool fused, cudaStream_t stream, const DeviceInfo& dev);
+// Tile configuration of one GEMM launch.
+struct GemmConfig {
+  int cta_group;  // 1: one CTA per 128-row tile; 2: CTA pairs with 256-row tiles
+  int tile_n;     // output tile width
+  int acc_bufs;   // accumulator buffers in TMEM
+};
+GemmConfig gemm_config(int64_t M, int64_t N);
+cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused,
+                        cudaStream_t stream, const DeviceInfo& dev);
 
 }  // namespace nvfp4
