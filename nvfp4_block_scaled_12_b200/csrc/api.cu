@@ -228,7 +228,10 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
   const DeviceInfo* dev = nullptr;
   nvfp4_status st = current_device(&dev);
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_quantize(x, M, K, g, codes, sf, static_cast<cudaStream_t>(stream), *dev);
+  CUtensorMap tx;
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_quantize(tx, M, K, g, codes, sf, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return ok();
 }

@@ -47,7 +47,8 @@ struct GemmTensorMaps {
   CUtensorMap y;         // bf16 destination of the plain or BF16-range epilogue
 };
 
-cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
+// tmap_x: bf16 [M, K], box 128 rows x 64 columns, 128-byte swizzle.
+cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
                             cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_calibrate(const void* x, int64_t n, float* out, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out, cudaStream_t stream);

@@ -3,11 +3,15 @@
 // "Kernels": `nvfp4_quantize` runs on the activations at every forward).
 //
 // The quantize kernel is HBM-bound (2 bytes read, 0.5 + 1/16 bytes written per
-// element).  Each CTA owns a 128-row x 128-column tile: the scales of such a
-// tile are exactly two 512-byte atoms of the swizzled scale layout, so they
-// are assembled in shared memory and written with full 16-byte stores.
-// Every thread issues all eight of its 16-byte loads before doing any math to
-// keep enough bytes in flight per SM.
+// element).  One persistent CTA per SM streams tiles of 128 rows x 64 columns
+// (16 KB of bf16, the width of one scale atom) through a 10-stage TMA ring in
+// shared memory (160 KB in flight per SM), loaded with the 128-byte swizzle so
+// that 32 threads reading 32 different rows hit distinct banks.  Sixteen
+// consumer warps work independently, with no block-wide barrier: four groups
+// of four warps take every fourth tile, and warp q of a group owns rows
+// 32q..32q+31 of it.  A thread owns one row's 64 elements (four 16-element
+// blocks), so it produces exactly one 4-byte word of the swizzled scale layout
+// and 32 bytes of codes.
 #include "internal.h"
 
 namespace nvfp4 {
@@ -15,69 +19,122 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kQRows = 128;
-constexpr int kQCols = 128;
-constexpr int kQThreads = 256;
-constexpr int kQLoads = kQRows * kQCols / 8 / kQThreads;  // 16-byte loads per thread (8)
+constexpr int kQCols = 64;
+constexpr int kQStages = 10;
+constexpr int kQGroups = 4;                         // tiles processed concurrently per CTA
+constexpr int kQConsumerWarps = 4 * kQGroups;       // 4 quarter-warps per tile
+constexpr int kQThreads = (kQConsumerWarps + 1) * 32;  // + one producer warp
+constexpr uint32_t kQTileBytes = kQRows * kQCols * 2;  // 16 KB of bf16
+constexpr uint32_t kQOffBar = kQStages * kQTileBytes;
+constexpr uint32_t kQSmemBytes = kQOffBar + 2 * kQStages * 8 + 16 + 1024;
 
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(const __nv_bfloat16* __restrict__ x, int64_t M,
-                                                             int64_t K, float g, uint8_t* __restrict__ codes,
-                                                             uint8_t* __restrict__ sf, int64_t tiles_k,
-                                                             int64_t n_tiles) {
-  __shared__ __align__(16) uint8_t sf_tile[2 * 512];
-  const int tid = threadIdx.x;
-  const int cg = tid & 15;    // 8-column group inside the tile
-  const int rsub = tid >> 4;  // first row of this thread (0..15), then +16 per load
-  const float d6 = __fmul_rn(6.0f, g);
-  const int64_t katoms = K >> 6;
-
-  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const int64_t row0 = (tile / tiles_k) * kQRows;
-    const int64_t col0 = (tile % tiles_k) * kQCols;
-    const int64_t col = col0 + cg * 8;
-    const bool col_ok = col < K;  // K % 64 == 0: 64-column halves are all-in or all-out
-
-    uint4 v[kQLoads];
-#pragma unroll
-    for (int i = 0; i < kQLoads; ++i) {
-      const int64_t row = row0 + rsub + 16 * i;
-      v[i] = (row < M && col_ok) ? ld_stream_v4(x + row * K + col) : make_uint4(0u, 0u, 0u, 0u);
+__global__ void __launch_bounds__(kQThreads, 1)
+    quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t M, int64_t K, float g,
+                    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int64_t tiles_k, int64_t n_tiles,
+                    unsigned* fault_word) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQOffBar);
+  uint64_t* empty = full + kQStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQStages);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);  // the four quarter-warps of the tile
     }
-
-#pragma unroll
-    for (int i = 0; i < kQLoads; ++i) {
-      const int rloc = rsub + 16 * i;
-      const int64_t row = row0 + rloc;
-      float f[8] = {bf16_lo(v[i].x), bf16_hi(v[i].x), bf16_lo(v[i].y), bf16_hi(v[i].y),
-                    bf16_lo(v[i].z), bf16_hi(v[i].z), bf16_lo(v[i].w), bf16_hi(v[i].w)};
-      float amax = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // partner holds the other 8
-      const uint32_t s = e4m3_from_f32_satfinite(__fdiv_rn(amax, d6));
-      uint32_t word = 0u;
-      if (s != 0u) {
-        const float r = __frcp_rn(__fmul_rn(e4m3_to_f32(s), g));
-        word = e2m1x8_from_f32(__fmul_rn(f[0], r), __fmul_rn(f[1], r), __fmul_rn(f[2], r),
-                               __fmul_rn(f[3], r), __fmul_rn(f[4], r), __fmul_rn(f[5], r),
-                               __fmul_rn(f[6], r), __fmul_rn(f[7], r));
-      }
-      if (row < M && col_ok) *reinterpret_cast<uint32_t*>(codes + row * (K >> 1) + (col >> 1)) = word;
-      if ((cg & 1) == 0) {
-        const int c = cg >> 1;  // scale column inside the tile, 0..7
-        sf_tile[(c >> 2) * 512 + (rloc & 31) * 16 + (rloc >> 5) * 4 + (c & 3)] = static_cast<uint8_t>(s);
-      }
-    }
-    __syncthreads();
-    if (tid < 64) {
-      const int atom = tid >> 5;
-      const int64_t katom = (col0 >> 6) + atom;
-      if (katom < katoms) {
-        const uint4 w = *reinterpret_cast<const uint4*>(sf_tile + tid * 16);
-        *reinterpret_cast<uint4*>(sf + ((row0 >> 7) * katoms + katom) * 512 + (tid & 31) * 16) = w;
-      }
-    }
-    __syncthreads();
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  __syncthreads();
+  unsigned fault = 0u;
+  // this CTA's tiles are blockIdx.x + j * gridDim.x, j = 0, 1, ...; local
+  // tile j lives in stage j % kQStages
+  const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+  if (warp == kQConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_x);
+      int64_t j = 0;
+      for (; j < my_tiles; ++j) {
+        const int stage = static_cast<int>(j % kQStages);
+        const uint32_t phase = static_cast<uint32_t>((j / kQStages) & 1);
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          fault = kFaultProducerWait;
+          break;
+        }
+        const int64_t tile = blockIdx.x + j * gridDim.x;
+        mbar_arrive_expect_tx(&full[stage], kQTileBytes);
+        tma_load_2d(smem + stage * kQTileBytes, &tmap_x, &full[stage], static_cast<int32_t>((tile % tiles_k) * kQCols),
+                    static_cast<int32_t>((tile / tiles_k) * kQRows));
+      }
+      if (fault != 0u) {
+        *abort_flag = 1;
+        // let the copies already issued (the last kQStages tiles) land
+        for (int64_t i = j - 1; i >= 0 && i >= j - kQStages; --i)
+          mbar_wait(&full[i % kQStages], static_cast<uint32_t>((i / kQStages) & 1), nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int group = warp >> 2;
+    const int q = warp & 3;         // rows 32q..32q+31 of each tile
+    const int rloc = q * 32 + lane; // this thread's row inside the tile
+    const float d6 = __fmul_rn(6.0f, g);
+    const int64_t katoms = K >> 6;
+    for (int64_t j = group; j < my_tiles; j += kQGroups) {
+      const int stage = static_cast<int>(j % kQStages);
+      const uint32_t phase = static_cast<uint32_t>((j / kQStages) & 1);
+      const bool got = mbar_wait(&full[stage], phase, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        fault = kFaultEpilogueWait;
+        break;
+      }
+      // row rloc: 128 bytes, 16-byte chunk c stored at chunk c ^ (rloc % 8)
+      const uint8_t* row_s = smem + stage * kQTileBytes + rloc * 128;
+      uint4 v[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(row_s + ((c ^ (rloc & 7)) * 16));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);  // this quarter is in registers
+
+      const int64_t tile = blockIdx.x + j * gridDim.x;
+      const int64_t row = (tile / tiles_k) * kQRows + rloc;
+      const int64_t katom = tile % tiles_k;  // 64-column group = scale atom column
+      uint32_t sfw = 0u;
+      uint32_t cw[8];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float f[16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 u = v[2 * b + h];
+          f[8 * h + 0] = bf16_lo(u.x);
+          f[8 * h + 1] = bf16_hi(u.x);
+          f[8 * h + 2] = bf16_lo(u.y);
+          f[8 * h + 3] = bf16_hi(u.y);
+          f[8 * h + 4] = bf16_lo(u.z);
+          f[8 * h + 5] = bf16_hi(u.z);
+          f[8 * h + 6] = bf16_lo(u.w);
+          f[8 * h + 7] = bf16_hi(u.w);
+        }
+        sfw |= quantize_block16(f, g, d6, cw[2 * b], cw[2 * b + 1]) << (8 * b);
+      }
+      if (row < M) {
+        uint8_t* crow = codes + row * (K >> 1) + katom * 32;
+        *reinterpret_cast<uint4*>(crow) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4*>(crow + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      }
+      // rows past M belong to the zero padding of the scale buffer (their
+      // data was zero-filled by the TMA, so sfw == 0)
+      *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 4, katoms)) = sfw;
+    }
+    if (fault != 0u) *abort_flag = 1;
+  }
+  if (fault != 0u && lane == 0 && fault_word != nullptr) atomicOr(fault_word, fault);
+  __syncthreads();
 }
 
 // One thread per 16-byte line of an atom: gathers rows r, r+32, r+64, r+96
@@ -106,15 +163,15 @@ __global__ void swizzle_sf_kernel(const uint8_t* __restrict__ sf_lin, int64_t ro
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
+cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
                             cudaStream_t stream, const DeviceInfo& dev) {
   const int64_t tiles_m = (M + kQRows - 1) / kQRows;
   const int64_t tiles_k = (K + kQCols - 1) / kQCols;
   const int64_t n_tiles = tiles_m * tiles_k;
-  const int64_t resident = static_cast<int64_t>(dev.num_sms) * 8;
-  const int grid = static_cast<int>(n_tiles < resident ? n_tiles : resident);
-  quantize_kernel<<<grid, kQThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), M, K, g, codes, sf,
-                                                  tiles_k, n_tiles);
+  const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
+  cudaError_t err = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+  if (err != cudaSuccess) return err;
+  quantize_kernel<<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles, dev.fault);
   return cudaGetLastError();
 }
 
