@@ -39,6 +39,37 @@ FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PFLOP/s FP4 vs 2.25 PFLOP/s bf16
 QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
 
 
+PROFILES = os.path.join(ROOT, "profiles")
+GEMM_PROFILE = os.path.join(PROFILES, "gemm_nvf4_flux_mlp_up_m4608_k3072_n12288.txt")
+GEMM_SOURCES = ("gemm.cu", "device.cuh", "internal.h")
+
+
+def gemm_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_12_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_dram_traffic():
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu
+    summary, or None when the kernel's sources changed since the capture."""
+    try:
+        fields = {}
+        with open(GEMM_PROFILE) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("sources_sha256") != gemm_sources_sha256():
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -117,6 +148,11 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def rank_activation_seed(rank: int, base_seed: int) -> int:
+    """Each rank draws its own token batch (weak scaling, no data exchange)."""
+    return base_seed + 100 * rank
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
@@ -241,7 +277,7 @@ def run_ours(args):
     M, K, N = wl.m, wl.k, wl.n
     flops = 2.0 * M * N * K
     # each rank gets its own token batch (independent seeds): weak scaling
-    x = synth.activations_with_outlier_channels(M, K, seed=wl.seed + 100 * rank).to(device)
+    x = synth.activations_with_outlier_channels(M, K, seed=rank_activation_seed(rank, wl.seed)).to(device)
     w = wl.weight().to(device)
     bias = wl.bias_vec().to(device)
     g_x = F.global_scale(x)              # calibrated input_scale (offline)
@@ -256,7 +292,7 @@ def run_ours(args):
         # lines of an unrelated buffer, so the timed kernels read their inputs
         # from HBM and do not pay for write-backs of the flush itself
         flush.zero_()
-        flush.sum()
+        flush.view(torch.int64).sum()
 
     def step():
         F.quantize(x, g_x, out=xq, stream=stream)
@@ -358,7 +394,7 @@ def run_ours(args):
                        "bias": True, "global_batch_tokens": world * M, "parallelism": f"dp{world} (token shards)",
                        "l2": "flushed between timed steps: 256 MiB written then read, outside the events"},
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak, "unit": "TFLOP/s",
-                         "frac": gemm_tf / fp4_peak, "traffic": None,
+                         "frac": gemm_tf / fp4_peak, "traffic": gemm_dram_traffic(),
                          "peak_source": f"{src} bf16 burst x {FP4_PER_BF16:g} (nominal FP4/bf16 dense ratio)"},
             "kernels": {
                 "gemm": {"ms": gemm_ms, "tflops": gemm_tf, "frac_of_fp4_peak": gemm_tf / fp4_peak},
