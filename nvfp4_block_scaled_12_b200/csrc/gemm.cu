@@ -10,10 +10,13 @@
 //            leader issues tcgen05.mma.cta_group::2 (M=256, N=192, K=64), so
 //            every B byte crosses L2 once per pair.  Used for M > 128.
 //   kCG = 1  one CTA owns a 128 x 192 tile (small M).
-// Warps (10 per CTA):
-//   0     TMA producer: A/B tiles (128-byte rows, 128-byte swizzle) and the
-//         scale atoms (3-D boxes, zero-filled past K and past the last row
-//         block) into a shared-memory ring.
+// Warps (11 per CTA):
+//   0, 10 TMA producers, alternating k-tiles: A/B tiles (128-byte rows,
+//         128-byte swizzle) and the scale atoms (3-D boxes, zero-filled past
+//         K and past the last row block) into a shared-memory ring.  A TMA
+//         instruction holds its issuing thread long enough that one thread
+//         cannot keep the SM's TMA unit busy; two issuing warps reach about
+//         twice the load rate.
 //   1     allocates TMEM; in the leader one thread issues the MMAs into a
 //         double-buffered fp32 accumulator.
 //   2-5   epilogue: tcgen05.ld 32 columns at a time, alpha*acc + bias, bf16,
@@ -43,7 +46,8 @@ namespace {
 constexpr int kBKBytes = 128;   // 256 fp4 elements per row per stage
 constexpr uint32_t kABytes = 128 * kBKBytes;  // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t kSfaBytes = 4 * 512;       // 4 k-blocks x one 128-row atom
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
+constexpr int kProducers = 2;  // warps 0 and 10
 constexpr uint32_t kTmemCols = 512;
 
 // kCG: CTAs per tile; kBN: tile width; kAcc: accumulator buffers in TMEM.
@@ -62,7 +66,10 @@ struct Cfg {
   static constexpr int kSfSlots = (kTmemCols - kSfCol) / kSfSlotCols > 8 ? 8 : (kTmemCols - kSfCol) / kSfSlotCols;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStagesFit = (224 * 1024 - 4 * 2 * 2048) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  // a multiple of the producer count: each stage then has a single producer
+  // (an mbarrier wait only tells phases apart by parity, so one waiter must
+  // see a stage's phases in order)
+  static constexpr int kStages = (kStagesFit > 8 ? 8 : kStagesFit) / kProducers * kProducers;
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
   static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
@@ -190,51 +197,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(bar);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------ producers
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int last_phase[S];
-#pragma unroll
-      for (int s = 0; s < S; ++s) last_phase[s] = -1;
-      for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
-        const int tm = tile % p.tiles_m;
-        const int n0 = (tile / p.tiles_m) * kBN;
-        const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
-        for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
-            fault = kFaultProducerWait;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
-          mbar_arrive_expect_tx(&sfin[stage], kSfaBytes + C::kSfbBytes);
-          uint8_t* sa = smem + C::kOffA + stage * kABytes;
-          uint8_t* sb = smem + C::kOffB + stage * C::kBBytes;
-          if (kCG == 2) {
-            const uint32_t fb = peer_smem(smem_u32(&full[stage]), 0);
-            tma_load_2d_pair(sa, &tmap_a, fb, kt * kBKBytes, row_block * 128);
-            tma_load_2d_pair(sb, &tmap_b, fb, kt * kBKBytes, n0 + static_cast<int>(rank) * C::kBNc);
-          } else {
-            tma_load_2d(sa, &tmap_a, &full[stage], kt * kBKBytes, row_block * 128);
-            tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
-          }
-          tma_load_3d(smem + C::kOffSfa + stage * kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * 4, row_block);
-          tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * 4, n0 >> 7);
-          last_phase[stage] = static_cast<int>(phase);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+      const int pid = warp == 0 ? 0 : 1;
+      if (pid == 0) {
+        // Every CTA first asks L2 for its 1/gridDim share of the operands: all
+        // of them fit in L2, and a stage whose rows include one first touch
+        // would otherwise wait the full DRAM latency.
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t share = ((p.pf_bytes[i] + gridDim.x - 1) / gridDim.x + 15) & ~uint64_t(15);
+          const uint64_t begin = share * blockIdx.x;
+          const uint64_t end = begin + share < p.pf_bytes[i] ? begin + share : p.pf_bytes[i];
+          for (uint64_t off = begin; off < end; off += 65536) {
+            const uint64_t n = end - off < 65536 ? end - off : 65536;
+            prefetch_l2_bulk(p.pf_ptr[i] + off, static_cast<uint32_t>(n));
           }
         }
       }
+      // flattened (tile, k-tile) sequence of this CTA group; producer pid
+      // issues the entries j with j % kProducers == pid into stage j % S
+      const int my_tiles = p.num_tiles > cluster ? (p.num_tiles - cluster + num_clusters - 1) / num_clusters : 0;
+      const int64_t total = static_cast<int64_t>(my_tiles) * p.num_kt;
+      int64_t j = pid;
+      for (; j < total; j += kProducers) {
+        const int stage = static_cast<int>(j % S);
+        const uint32_t phase = static_cast<uint32_t>((j / S) & 1);
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          fault = kFaultProducerWait;
+          break;
+        }
+        const int tile = cluster + static_cast<int>(j / p.num_kt) * num_clusters;
+        const int kt = static_cast<int>(j % p.num_kt);
+        const int tm = tile % p.tiles_m;
+        const int n0 = (tile / p.tiles_m) * kBN;
+        const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
+        if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
+        mbar_arrive_expect_tx(&sfin[stage], kSfaBytes + C::kSfbBytes);
+        uint8_t* sa = smem + C::kOffA + stage * kABytes;
+        uint8_t* sb = smem + C::kOffB + stage * C::kBBytes;
+        if (kCG == 2) {
+          const uint32_t fb = peer_smem(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(sa, &tmap_a, fb, kt * kBKBytes, row_block * 128);
+          tma_load_2d_pair(sb, &tmap_b, fb, kt * kBKBytes, n0 + static_cast<int>(rank) * C::kBNc);
+        } else {
+          tma_load_2d(sa, &tmap_a, &full[stage], kt * kBKBytes, row_block * 128);
+          tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
+        }
+        tma_load_3d(smem + C::kOffSfa + stage * kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * 4, row_block);
+        tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * 4, n0 >> 7);
+      }
       if (fault != 0u) {
         *abort_flag = 1;
-        // let every copy already issued land before shared memory goes away
-        for (int s = 0; s < S; ++s) {
-          if (last_phase[s] < 0) continue;
-          mbar_wait(&sfin[s], static_cast<uint32_t>(last_phase[s]), nullptr);
-          if (leader) mbar_wait(&full[s], static_cast<uint32_t>(last_phase[s]), nullptr);
+        // let the copies this producer issued (its last S / kProducers entries) land
+        for (int64_t i = j - kProducers; i >= 0 && i >= j - S; i -= kProducers) {
+          const int stage = static_cast<int>(i % S);
+          const uint32_t phase = static_cast<uint32_t>((i / S) & 1);
+          mbar_wait(&sfin[stage], phase, nullptr);
+          if (leader) mbar_wait(&full[stage], phase, nullptr);
         }
       }
     }
@@ -305,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 6) {
-    // ------------------------------------------------------------ scale movers
+    // ------------------------------------------------------------ scale movers (warps 6-9)
     const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter of this warp
     int stage = 0;
     uint32_t phase = 0;

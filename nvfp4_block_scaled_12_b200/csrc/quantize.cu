@@ -4,12 +4,15 @@
 //
 // The quantize kernel is HBM-bound (2 bytes read, 0.5 + 1/16 bytes written per
 // element).  One persistent CTA per SM streams tiles of 128 rows x 64 columns
-// (16 KB of bf16, the width of one scale atom) through a 10-stage TMA ring in
-// shared memory (160 KB in flight per SM), loaded with the 128-byte swizzle so
+// (16 KB of bf16, the width of one scale atom) through 12 TMA stages in
+// shared memory (192 KB in flight per SM), loaded with the 128-byte swizzle so
 // that 32 threads reading 32 different rows hit distinct banks.  Sixteen
 // consumer warps work independently, with no block-wide barrier: four groups
 // of four warps take every fourth tile, and warp q of a group owns rows
-// 32q..32q+31 of it.  A thread owns one row's 64 elements (four 16-element
+// 32q..32q+31 of it.  Each group has its own three stages: an mbarrier wait
+// only tells phases apart by parity, so a stage must be consumed in order by
+// one consumer (a group running ahead on a shared ring could take a stage's
+// previous phase for its next one).  A thread owns one row's 64 elements (four 16-element
 // blocks), so it produces exactly one 4-byte word of the swizzled scale layout
 // and 32 bytes of codes.
 #include "internal.h"
@@ -20,8 +23,9 @@ namespace {
 
 constexpr int kQRows = 128;
 constexpr int kQCols = 64;
-constexpr int kQStages = 10;
 constexpr int kQGroups = 4;                         // tiles processed concurrently per CTA
+constexpr int kQStagesPerGroup = 3;
+constexpr int kQStages = kQGroups * kQStagesPerGroup;
 constexpr int kQConsumerWarps = 4 * kQGroups;       // 4 quarter-warps per tile
 constexpr int kQThreads = (kQConsumerWarps + 1) * 32;  // + one producer warp
 constexpr uint32_t kQTileBytes = kQRows * kQCols * 2;  // 16 KB of bf16
@@ -50,7 +54,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   __syncthreads();
   unsigned fault = 0u;
   // this CTA's tiles are blockIdx.x + j * gridDim.x, j = 0, 1, ...; local
-  // tile j lives in stage j % kQStages
+  // tile j = 4i + g goes to group g, stage g * kQStagesPerGroup + i % 3
   const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
   if (warp == kQConsumerWarps) {
@@ -59,8 +63,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       prefetch_tmap(&tmap_x);
       int64_t j = 0;
       for (; j < my_tiles; ++j) {
-        const int stage = static_cast<int>(j % kQStages);
-        const uint32_t phase = static_cast<uint32_t>((j / kQStages) & 1);
+        const int64_t i = j / kQGroups;
+        const int stage = static_cast<int>(j % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
+        const uint32_t phase = static_cast<uint32_t>((i / kQStagesPerGroup) & 1);
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
           fault = kFaultProducerWait;
           break;
@@ -73,8 +78,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (fault != 0u) {
         *abort_flag = 1;
         // let the copies already issued (the last kQStages tiles) land
-        for (int64_t i = j - 1; i >= 0 && i >= j - kQStages; --i)
-          mbar_wait(&full[i % kQStages], static_cast<uint32_t>((i / kQStages) & 1), nullptr);
+        for (int64_t jj = j - 1; jj >= 0 && jj >= j - kQStages; --jj) {
+          const int64_t i = jj / kQGroups;
+          const int stage = static_cast<int>(jj % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
+          mbar_wait(&full[stage], static_cast<uint32_t>((i / kQStagesPerGroup) & 1), nullptr);
+        }
       }
     }
   } else {
@@ -85,8 +93,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const float d6 = __fmul_rn(6.0f, g);
     const int64_t katoms = K >> 6;
     for (int64_t j = group; j < my_tiles; j += kQGroups) {
-      const int stage = static_cast<int>(j % kQStages);
-      const uint32_t phase = static_cast<uint32_t>((j / kQStages) & 1);
+      const int64_t i = j / kQGroups;
+      const int stage = group * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
+      const uint32_t phase = static_cast<uint32_t>((i / kQStagesPerGroup) & 1);
       const bool got = mbar_wait(&full[stage], phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         fault = kFaultEpilogueWait;
@@ -97,6 +106,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
       uint4 v[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(row_s + ((c ^ (rloc & 7)) * 16));
+      // The stage is refilled by TMA (the async proxy) once all four warps
+      // have arrived: order this thread's shared-memory reads before that
+      // write, or a load still in flight can return the next tile's data.
+      fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);  // this quarter is in registers
 
