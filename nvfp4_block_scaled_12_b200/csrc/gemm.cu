@@ -17,23 +17,26 @@
 //         instruction holds its issuing thread long enough that one thread
 //         cannot keep the SM's TMA unit busy; two issuing warps reach about
 //         twice the load rate.
-//   1     allocates TMEM; in the leader one thread issues the MMAs into a
-//         double-buffered fp32 accumulator.
+//   1     allocates TMEM; in the leader one thread waits for one barrier per
+//         k-tile, issues the MMAs into a double-buffered fp32 accumulator and
+//         commits once: that commit frees the shared-memory stage and the
+//         TMEM scale slot of the k-tile together.
 //   2-5   epilogue: tcgen05.ld 32 columns at a time, alpha*acc + bias, bf16,
 //         swizzled staging in shared memory, TMA store (or the fused
 //         quantize); drains accumulator i while the MMA fills i^1.
 //   6-9   scale movers: copy each stage's scale atoms from shared memory into
-//         a double-buffered TMEM slot with tcgen05.st, one warp per 32-lane
-//         TMEM quarter.  The MMA reads every scale row from all four quarters,
-//         so each quarter holds a full copy.  Register-path stores run beside
-//         the tensor pipe, where tcgen05.cp copies of the same (replicated)
-//         data would serialize with the MMAs.
-// TMEM columns: [0,192) and [192,384) accumulators; [384,432) and [432,480)
-// scale slots, each 16 columns of A scales (4 per MMA k-block) then 32 of B
-// scales (8 per k-block, covering two 128-row atom blocks).  Scale column j
-// of lane l holds the 4 scales of row 32*j + l, so row i of a tile is read
-// from column i/32; a 192-wide B tile that starts at row 64 of a 128-row atom
-// block skips 2 columns.
+//         a ring of TMEM slots with tcgen05.st, one warp per 32-lane TMEM
+//         quarter, and arrive on the same barrier as the A/B bytes.  The MMA
+//         reads every scale row from all four quarters, so each quarter holds
+//         a full copy.  Register-path stores run beside the tensor pipe, where
+//         tcgen05.cp copies of the same (replicated) data would serialize with
+//         the MMAs.
+// TMEM columns: the accumulators first, then the scale slots: 16 columns of A
+// scales each (4 per MMA k-block), then kBN/8 columns of B scales each
+// (kBN/32 per k-block).  Scale column j of lane l holds the 4 scales of row
+// 32*j + l, so row i of a tile is read from column i/32; the movers pick the
+// kBN/32 row groups of the tile out of the 128-row atom blocks it touches (a
+// 192-wide tile may start at row 64 of a block).
 // Every barrier wait is bounded (see mbar_wait); a role that gives up sets
 // the CTA's abort flag and the device fault word, lets the copies it issued
 // land, and the CTA still reaches the final barrier and frees its TMEM.
@@ -59,32 +62,38 @@ struct Cfg {
   // 128-row scale blocks a B tile can touch (a 192-wide tile may start mid-block)
   static constexpr int kSfbBlocks = kBN % 128 == 0 ? kBN / 128 : kBN / 128 + 1;
   static constexpr uint32_t kSfbBytes = kSfbBlocks * 4 * 512;
-  // TMEM: accumulators, then a ring of per-k-tile scale slots
-  static constexpr uint32_t kSfCol = kAcc * kBN;
-  static constexpr uint32_t kSfbOff = 16;  // 16 A-scale columns, then 4 per B block per k-block
-  static constexpr uint32_t kSfSlotCols = 16 + 16 * kSfbBlocks;
-  static constexpr int kSfSlots = (kTmemCols - kSfCol) / kSfSlotCols > 8 ? 8 : (kTmemCols - kSfCol) / kSfSlotCols;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStagesFit = (224 * 1024 - 4 * 2 * 2048) / kStageBytes;
   // a multiple of the producer count: each stage then has a single producer
   // (an mbarrier wait only tells phases apart by parity, so one waiter must
   // see a stage's phases in order)
   static constexpr int kStages = (kStagesFit > 8 ? 8 : kStagesFit) / kProducers * kProducers;
+  // TMEM: accumulators, then the scale slots.  Slot j % kSfSlots holds the
+  // scales of k-tile j; the movers refill it once the commit of k-tile
+  // j - kSfSlots has arrived on that k-tile's empty barrier, which can only
+  // be the phase they wait for while kSfSlots <= kStages.
+  static constexpr uint32_t kSfbGroups = kBN / 32;       // 32-row groups of B scales per k-block
+  static constexpr uint32_t kSfbSlotCols = 4 * kSfbGroups;
+  static constexpr int kSfSlotsFit = (kTmemCols - kAcc * kBN) / (16 + kSfbSlotCols);
+  static constexpr int kSfSlots = kSfSlotsFit < kStages ? (kSfSlotsFit > 8 ? 8 : kSfSlotsFit) : kStages;
+  static constexpr uint32_t kSfaCol = kAcc * kBN;
+  static constexpr uint32_t kSfbCol = kSfaCol + 16 * kSfSlots;
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
   static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
   static constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
   static constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;  // 4 warps x 2 x 2 KB
   static constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * 2048;
-  // full, empty, sfin per stage; acc_full, acc_empty per accumulator;
-  // sf_full, sf_empty per scale slot; drain
-  static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAcc + 2 * kSfSlots + 1;
+  // full, empty, sfin per stage; acc_full, acc_empty per accumulator; drain
+  static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAcc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kFullTx = kCG * (kABytes + kBBytes);  // A/B bytes of the whole group
   static_assert(kBN % 32 == 0 && kBN / kCG % 8 == 0, "tile width");
   static_assert(kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
-  static_assert(kSfSlots >= 2, "TMEM budget");
+  static_assert(kSfSlots >= 2 && kSfSlots <= kStages, "TMEM budget");
+  static_assert(kSfaCol % 16 == 0 && kSfbCol % 8 == 0 && kSfbSlotCols % 8 == 0, "tcgen05.st column alignment");
+  static_assert(kSfbCol + kSfSlots * kSfbSlotCols <= kTmemCols, "TMEM budget");
   static_assert(kStages >= 3, "pipeline depth");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -128,14 +137,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* full = bars;            // leader: A/B of the whole group landed
-  uint64_t* empty = bars + S;       // this CTA's stage may be refilled
+  uint64_t* full = bars;            // leader: A/B of the whole group landed, scales in TMEM
+  uint64_t* empty = bars + S;       // this CTA's stage and the k-tile's scale slot may be refilled
   uint64_t* sfin = bars + 2 * S;    // this CTA's scale atoms landed
   uint64_t* acc_full = bars + 3 * S;
   uint64_t* acc_empty = acc_full + kAcc;   // leader
-  uint64_t* sf_full = acc_empty + kAcc;    // leader
-  uint64_t* sf_empty = sf_full + R;
-  uint64_t* drain = sf_empty + R;
+  uint64_t* drain = acc_empty + kAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -148,17 +155,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 4 * kCG);  // the producer's expect_tx and every scale mover of the group
       mbar_init(&empty[s], 1);
       mbar_init(&sfin[s], 1);
     }
     for (int a = 0; a < kAcc; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 4 * kCG);
-    }
-    for (int r = 0; r < R; ++r) {
-      mbar_init(&sf_full[r], 4 * kCG);
-      mbar_init(&sf_empty[r], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -265,12 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int slot = 0;
-      uint32_t slot_phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
-        const int n0 = (tile / p.tiles_m) * kBN;
-        const uint32_t sfb_shift = (n0 & 127) ? 2u : 0u;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
           fault = kFaultMmaWait;
           break;
@@ -278,8 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag) ||
-              !mbar_wait(&sf_full[slot], slot_phase, abort_flag)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
             fault = kFaultMmaWait;
             break;
           }
@@ -287,26 +286,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nkb = min(4, p.k64 - kt * 4);
           const uint32_t sa = smem_u32(smem + C::kOffA + stage * kABytes);
           const uint32_t sb = smem_u32(smem + C::kOffB + stage * C::kBBytes);
-          const uint32_t sf = tmem_base + C::kSfCol + static_cast<uint32_t>(slot) * C::kSfSlotCols;
+          const uint32_t sfa = tmem_base + C::kSfaCol + static_cast<uint32_t>(slot) * 16u;
+          const uint32_t sfb = tmem_base + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols;
           for (int kb = 0; kb < nkb; ++kb) {
             const uint64_t ad = sdesc_kmajor_sw128(sa + kb * 32), bd = sdesc_kmajor_sw128(sb + kb * 32);
             const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
-            const uint32_t sfb = sf + C::kSfbOff + kb * 4 * C::kSfbBlocks + sfb_shift;
             if (kCG == 2)
-              tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, sf + kb * 4, sfb, accum);
+              tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
             else
-              tc_mma_nvf4(d_tmem, ad, bd, idesc, sf + kb * 4, sfb, accum);
+              tc_mma_nvf4(d_tmem, ad, bd, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
           }
-          commit_group(&empty[stage]);    // frees the smem stages once these MMAs have read them
-          commit_group(&sf_empty[slot]);  // and the scale slots
+          // frees the smem stage and the scale slot once these MMAs have read them
+          commit_group(&empty[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
-          if (++slot == R) {
-            slot = 0;
-            slot_phase ^= 1u;
-          }
+          if (++slot == R) slot = 0;
         }
         if (fault != 0u) break;
         commit_group(&acc_full[acc]);  // accumulators ready for both epilogues
@@ -327,48 +323,74 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 6) {
     // ------------------------------------------------------------ scale movers (warps 6-9)
     const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter of this warp
+    const uint32_t t_quarter = tmem_base + ((q * 32u) << 16);
     int stage = 0;
     uint32_t phase = 0;
+    int lag_stage = 0;  // stage and phase of k-tile j - R, whose commit frees slot j % R
+    uint32_t lag_phase = 0;
     int slot = 0;
-    uint32_t slot_phase = 0;
+    int64_t j = 0;
     for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
-      for (int kt = 0; kt < p.num_kt; ++kt) {
-        const bool got = mbar_wait(&sfin[stage], phase, abort_flag) &&
-                         mbar_wait(&sf_empty[slot], slot_phase ^ 1u, abort_flag);
+      // a 192-wide tile that starts at row 64 of a 128-row scale block
+      const bool mid = ((tile / p.tiles_m) * kBN & 127) != 0;
+      for (int kt = 0; kt < p.num_kt; ++kt, ++j) {
+        bool got = mbar_wait(&sfin[stage], phase, abort_flag);
+        if (got && j >= R) {
+          got = mbar_wait(&empty[lag_stage], lag_phase, abort_flag);
+          if (++lag_stage == S) {
+            lag_stage = 0;
+            lag_phase ^= 1u;
+          }
+        }
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
           fault = kFaultMmaWait;
           break;
         }
         tc_fence_after();
-        const int nkb = min(4, p.k64 - kt * 4);
+        // All loads first (atoms past K arrived zero-filled), then a few wide
+        // stores: a shared load is not reordered across a tcgen05.st.
         const uint8_t* ssfa = smem + C::kOffSfa + stage * kSfaBytes + lane * 16;
         const uint8_t* ssfb = smem + C::kOffSfb + stage * C::kSfbBytes + lane * 16;
-        const uint32_t t =
-            tmem_base + ((q * 32u) << 16) + C::kSfCol + static_cast<uint32_t>(slot) * C::kSfSlotCols;
-        for (int kb = 0; kb < nkb; ++kb) {
-          const uint4 a = *reinterpret_cast<const uint4*>(ssfa + kb * 512);
-          tmem_st_32x32b_x4(t + kb * 4, a);
-          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512);
-          if (C::kSfbBlocks == 2) {
-            const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 4 * 512 + kb * 512);
-            tmem_st_32x32b_x8(t + C::kSfbOff + kb * 8, b0, b1);
-          } else {
-            tmem_st_32x32b_x4(t + C::kSfbOff + kb * 4, b0);
+        uint32_t sa[16];
+        uint32_t sb[4 * C::kSfbGroups];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512);
+          sa[4 * kb + 0] = v.x;
+          sa[4 * kb + 1] = v.y;
+          sa[4 * kb + 2] = v.z;
+          sa[4 * kb + 3] = v.w;
+          uint32_t w[4 * C::kSfbBlocks];
+#pragma unroll
+          for (int blk = 0; blk < C::kSfbBlocks; ++blk) {
+            const uint4 u = *reinterpret_cast<const uint4*>(ssfb + blk * 4 * 512 + kb * 512);
+            w[4 * blk + 0] = u.x;
+            w[4 * blk + 1] = u.y;
+            w[4 * blk + 2] = u.z;
+            w[4 * blk + 3] = u.w;
+          }
+#pragma unroll
+          for (int g = 0; g < static_cast<int>(C::kSfbGroups); ++g) {
+            if constexpr (kBN % 128 != 0)
+              sb[kb * C::kSfbGroups + g] = mid ? w[g + 2] : w[g];
+            else
+              sb[kb * C::kSfbGroups + g] = w[g];
           }
         }
+        tmem_st_32x32b_x16(t_quarter + C::kSfaCol + static_cast<uint32_t>(slot) * 16u, sa);
+#pragma unroll
+        for (int c = 0; c < static_cast<int>(C::kSfbSlotCols / 8); ++c)
+          tmem_st_32x32b_x8(t_quarter + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols + c * 8, sb + 8 * c);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(&sf_full[slot]);
+        if (lane == 0) arrive_leader(&full[stage]);
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
-        if (++slot == R) {
-          slot = 0;
-          slot_phase ^= 1u;
-        }
+        if (++slot == R) slot = 0;
       }
     }
     if (fault != 0u) *abort_flag = 1;
