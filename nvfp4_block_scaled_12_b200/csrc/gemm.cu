@@ -288,13 +288,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sb = smem_u32(smem + C::kOffB + stage * C::kBBytes);
           const uint32_t sfa = tmem_base + C::kSfaCol + static_cast<uint32_t>(slot) * 16u;
           const uint32_t sfb = tmem_base + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols;
-          for (int kb = 0; kb < nkb; ++kb) {
-            const uint64_t ad = sdesc_kmajor_sw128(sa + kb * 32), bd = sdesc_kmajor_sw128(sb + kb * 32);
-            const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
-            if (kCG == 2)
-              tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
-            else
-              tc_mma_nvf4(d_tmem, ad, bd, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
+          // One thread issues the MMAs and the tensor pipe queues few of them,
+          // so the instructions between two MMAs are on the critical path: the
+          // full k-tile takes a straight-line path with every operand address
+          // formed up front (a descriptor's start address field counts 16-byte
+          // units, so the next 32-byte k-block is +2).
+          const uint64_t ad = sdesc_kmajor_sw128(sa), bd = sdesc_kmajor_sw128(sb);
+          if (nkb == 4) {
+            const uint32_t first = kt != 0 ? 1u : 0u;
+            if (kCG == 2) {
+              tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, sfa, sfb, first);
+              tc_mma_nvf4_pair(d_tmem, ad + 2, bd + 2, idesc, sfa + 4, sfb + C::kSfbGroups, 1u);
+              tc_mma_nvf4_pair(d_tmem, ad + 4, bd + 4, idesc, sfa + 8, sfb + 2 * C::kSfbGroups, 1u);
+              tc_mma_nvf4_pair(d_tmem, ad + 6, bd + 6, idesc, sfa + 12, sfb + 3 * C::kSfbGroups, 1u);
+            } else {
+              tc_mma_nvf4(d_tmem, ad, bd, idesc, sfa, sfb, first);
+              tc_mma_nvf4(d_tmem, ad + 2, bd + 2, idesc, sfa + 4, sfb + C::kSfbGroups, 1u);
+              tc_mma_nvf4(d_tmem, ad + 4, bd + 4, idesc, sfa + 8, sfb + 2 * C::kSfbGroups, 1u);
+              tc_mma_nvf4(d_tmem, ad + 6, bd + 6, idesc, sfa + 12, sfb + 3 * C::kSfbGroups, 1u);
+            }
+          } else {
+            for (int kb = 0; kb < nkb; ++kb) {
+              const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
+              if (kCG == 2)
+                tc_mma_nvf4_pair(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
+              else
+                tc_mma_nvf4(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
+            }
           }
           // frees the smem stage and the scale slot once these MMAs have read them
           commit_group(&empty[stage]);
