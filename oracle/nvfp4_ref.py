@@ -43,6 +43,11 @@ Pins (the tests that tie each function to something other than itself):
   quantize_nvfp4                 tests/test_oracle_quant.py (round trip of
                                  representable blocks, zero blocks, saturation,
                                  brute-force nearest code)
+  dynamic_scale / quantize_dynamic
+                                 tests/test_oracle_quant.py (power-of-two
+                                 closed forms, the tensor's largest element
+                                 lands on code +-6 under scale 448, all-zero
+                                 tensor, both clamps)
   swizzle_sf / sf_offset         tests/test_oracle_quant.py (bijection, and an
                                  independent reshape/transpose construction)
   gemm_ref / dequantize          tests/test_oracle_gemm.py (closed form,
@@ -167,6 +172,40 @@ def global_scale(amax) -> np.float32:
 def tensor_amax(x) -> np.float32:
     """Largest magnitude of a float tensor (exact)."""
     return np.float32(np.max(np.abs(np.asarray(x, dtype=np.float32))))
+
+
+#: Range of per-tensor scales the quantizer accepts (the library's contract).
+G_MIN = np.float32(2.0 ** -64)
+G_MAX = np.float32(2.0 ** 64)
+
+
+def dynamic_scale(x):
+    """Per-tensor scale measured on the activation itself, for a layer that
+    has no calibrated ``input_scale`` (the BFL doc's ``nvfp4`` bullet makes the
+    calibrated scale the default; measuring it per call is the variant).
+
+    Returns ``(amax, g)``: ``amax = max |x|`` and ``g = amax / (6 * 448)``
+    (one fp32 division, as for a calibrated scale), clamped into
+    ``[G_MIN, G_MAX]``; ``g = 0`` when the tensor is all zeros.
+    """
+    amax = tensor_amax(x)
+    if amax == 0:
+        return amax, np.float32(0.0)
+    g = global_scale(amax)
+    return amax, np.float32(min(max(g, G_MIN), G_MAX))
+
+
+def quantize_dynamic(x):
+    """``quantize_nvfp4`` with the scale from ``dynamic_scale``; an all-zero
+    tensor (``g = 0``) gives all-zero codes and scales.
+    Returns ``(codes, sf, amax, g)``."""
+    x = np.asarray(x, dtype=np.float32)
+    amax, g = dynamic_scale(x)
+    if g == 0:
+        rows, K = x.shape
+        return np.zeros((rows, K // 2), np.uint8), np.zeros((rows, K // BLOCK), np.uint8), amax, g
+    codes, sf = quantize_nvfp4(x, g)
+    return codes, sf, amax, g
 
 
 # ----------------------------------------------------------------------------

@@ -172,6 +172,51 @@ def test_quantization_error_bound():
 
 
 # --------------------------------------------------------------------------
+# Dynamic (measured) per-tensor scale
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("k", [-20, -3, 0, 7, 40])
+def test_dynamic_scale_closed_form_for_power_of_two_amax(k):
+    # amax = 6 * 448 * 2^k is a bf16 value (21 * 2^(7+k)), so g = 2^k exactly.
+    rng = np.random.default_rng(k + 50)
+    x = O.round_to_bf16(rng.uniform(-1, 1, (64, 128)) * 2688.0 * 2.0 ** k).astype(np.float32)
+    x[17, 33] = -2688.0 * 2.0 ** k
+    amax, g = O.dynamic_scale(x)
+    assert amax == np.float32(2688.0 * 2.0 ** k)
+    assert g == np.float32(2.0 ** k)
+
+
+def test_dynamic_scale_puts_the_largest_element_on_the_top_code():
+    # The tensor's largest element sits at the top of both formats: its block
+    # scale is the largest E4M3 value (448, byte 0x7E) and its code is +-6.
+    rng = np.random.default_rng(51)
+    for trial in range(40):
+        x = O.round_to_bf16(rng.laplace(size=(32, 256)) * 10.0 ** rng.uniform(-6, 6)).astype(np.float32)
+        codes, sf, amax, g = O.quantize_dynamic(x)
+        r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+        assert sf[r, c // 16] == 0x7E
+        q = O.unpack_codes(codes)[r, c]
+        assert q == (0x7 if x[r, c] > 0 else 0xF)
+
+
+def test_dynamic_scale_of_an_all_zero_tensor_is_zero_and_output_is_zero():
+    x = np.zeros((8, 64), np.float32)
+    x[3, 5] = -0.0
+    codes, sf, amax, g = O.quantize_dynamic(x)
+    assert amax == 0 and g == 0
+    assert not codes.any() and not sf.any()
+
+
+def test_dynamic_scale_is_clamped_into_the_accepted_range():
+    tiny = np.full((4, 64), 2.0 ** -100, np.float32)   # amax / 2688 < 2^-64
+    huge = np.full((4, 64), 2.0 ** 120, np.float32)    # amax / 2688 > 2^64
+    assert O.dynamic_scale(tiny)[1] == O.G_MIN
+    assert O.dynamic_scale(huge)[1] == O.G_MAX
+    mid = np.full((4, 64), 2688.0 * 2.0 ** -64, np.float32)
+    assert O.dynamic_scale(mid)[1] == O.G_MIN          # the boundary itself is kept
+
+
+# --------------------------------------------------------------------------
 # Scale-factor swizzle
 # --------------------------------------------------------------------------
 
