@@ -371,6 +371,33 @@ def run_ours(args):
     ql_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ql_ev[3:]), world, device)
     F.nvfp4_check_fault()
 
+    # the dynamic-scale variant (per-tensor scale measured in the same
+    # launch): its quantize alone, on both shapes, and the MLP-up linear
+    # layer built on it (quantize_dynamic + GEMM reading g on the device)
+    ws = torch.empty(F.NVFP4_DYNAMIC_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+    xq_dyn = F.quantize_dynamic(x, workspace=ws, stream=stream)
+    xlq_dyn = F.quantize_dynamic(xl, workspace=ws, stream=stream)
+
+    def median_ms(fn, n=20, skip=3):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in evs:
+            flush_l2()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(device)
+        return max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs[skip:]), world, device)
+
+    qd_ms = median_ms(lambda: F.quantize_dynamic(x, out=xq_dyn, workspace=ws, stream=stream))
+    qdl_ms = median_ms(lambda: F.quantize_dynamic(xl, out=xlq_dyn, workspace=ws, stream=stream))
+
+    def linear_dynamic():
+        F.quantize_dynamic(x, out=xq_dyn, workspace=ws, stream=stream)
+        F.gemm(xq_dyn, wq, bias=bias, y=y, stream=stream)
+
+    ld_ms = median_ms(linear_dynamic)
+    F.nvfp4_check_fault()
+
     if rank == 0:
         hbm, bf16, src = peaks()
         fp4_peak = bf16 * FP4_PER_BF16
@@ -404,6 +431,19 @@ def run_ours(args):
                     "ms": ql_ms, "gbs": xl.numel() * QUANT_BYTES_PER_ELEM / (ql_ms * 1e-3) / 1e9,
                     "frac_of_hbm": xl.numel() * QUANT_BYTES_PER_ELEM / (ql_ms * 1e-3) / 1e9 / hbm,
                     "note": "standalone quantize workload (Laplace, spikes, zero blocks), median of 17, L2 flushed"},
+                "quantize_dynamic": {
+                    "ms": qd_ms, "gbs": M * K * QUANT_BYTES_PER_ELEM / (qd_ms * 1e-3) / 1e9,
+                    "frac_of_hbm": M * K * QUANT_BYTES_PER_ELEM / (qd_ms * 1e-3) / 1e9 / hbm,
+                    "note": "MLP-up activations with the scale measured in the same cooperative launch (amax pass, "
+                            "grid-wide max, quantize pass mostly from L2); bytes counted once, 2.5625 B/elem; "
+                            "median of 17, L2 flushed"},
+                "quantize_dynamic_4608x12288": {
+                    "ms": qdl_ms, "gbs": xl.numel() * QUANT_BYTES_PER_ELEM / (qdl_ms * 1e-3) / 1e9,
+                    "frac_of_hbm": xl.numel() * QUANT_BYTES_PER_ELEM / (qdl_ms * 1e-3) / 1e9 / hbm,
+                    "note": "standalone quantize workload, scale measured in the same launch; median of 17"},
+                "linear_dynamic": {
+                    "ms": ld_ms, "tflops": flops / (ld_ms * 1e-3) / 1e12,
+                    "note": "MLP-up step with the measured scale: quantize_dynamic + GEMM reading g on the device"},
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},

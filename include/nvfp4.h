@@ -113,6 +113,37 @@ nvfp4_status nvfp4_calibrate(const void* x, int64_t n, float* out, void* stream)
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g,
                             uint8_t* codes, uint8_t* sf, void* stream);
 
+/* Bytes of caller workspace one nvfp4_quantize_dynamic call uses. */
+#define NVFP4_DYNAMIC_WORKSPACE_BYTES 8
+
+/*
+ * Runtime activation quantization with the per-tensor scale measured on the
+ * activation itself, for a layer that has no calibrated `input_scale` (BFL
+ * doc, `nvfp4` bullet: the calibrated fp32 activation scale is the default;
+ * measuring it per call is the variant).  In one launch:
+ *     amax = max |x_i| over the whole tensor (exact)
+ *     g    = 0                                   if amax == 0
+ *            min(max(fl(amax / 2688), 2^-64), 2^64)  otherwise
+ *     codes, sf = nvfp4_quantize(x, g)   (all zero when g == 0)
+ *   x, M, K, codes, sf  as nvfp4_quantize.
+ *   scale_out  2 device floats (4-byte aligned), written: [0] = amax,
+ *              [1] = g (pass &scale_out[1] to nvfp4_gemm_dynamic).
+ *   workspace  device memory of at least NVFP4_DYNAMIC_WORKSPACE_BYTES
+ *              (4-byte aligned) that no other work uses while the call
+ *              runs; its contents on entry do not matter (the call zeroes
+ *              it on the stream before the kernel), on exit they are
+ *              unspecified.
+ * The kernel is a cooperative launch of at most one CTA per SM: every CTA
+ * folds its own tiles' maximum into the grid-wide one, then quantizes its
+ * tiles once all CTAs have arrived (a bounded wait: on time-out the kernel
+ * writes nothing more and records NVFP4_ETIMEOUT in the fault word).
+ * Errors: EINVAL (sizes, null, workspace too small), EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K,
+                                    uint8_t* codes, uint8_t* sf, float* scale_out,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 /*
  * Weight preparation: scatter ModelOpt's row-major E4M3 `weight_scale`
  * [rows, k/16] into the swizzled layout the GEMM reads (a byte permutation;
@@ -143,6 +174,21 @@ nvfp4_status nvfp4_swizzle_sf(const uint8_t* sf_linear, int64_t rows, int64_t k,
 nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                         const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
                         float alpha, const void* bias, void* y, void* stream);
+
+/*
+ * nvfp4_gemm for an activation whose per-tensor scale was measured on the
+ * device (nvfp4_quantize_dynamic): the epilogue reads g_a from device memory
+ * and uses alpha = fl(g_a[0] * g_b) (the same single fp32 product as
+ * input_scale * weight_scale_2).
+ *   g_a  device pointer to one float (4-byte aligned), read by the kernel;
+ *        work earlier on `stream` may write it.
+ *   g_b  the weight's per-tensor scale (weight_scale_2), finite.
+ * Other arguments and errors as nvfp4_gemm.
+ */
+nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                                float g_b, const float* g_a, const void* bias, void* y,
+                                void* stream);
 
 /* One column range of the fused epilogue. */
 typedef struct nvfp4_colrange {

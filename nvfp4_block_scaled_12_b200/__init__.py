@@ -25,6 +25,7 @@ NVFP4_OK, NVFP4_EINVAL, NVFP4_EALIGN, NVFP4_EARCH, NVFP4_ECUDA, NVFP4_ETIMEOUT =
 ACT_NONE, ACT_GELU_TANH = 0, 1
 DST_BF16, DST_NVFP4 = 0, 1
 MAX_RANGES = 8
+NVFP4_DYNAMIC_WORKSPACE_BYTES = 8
 
 _STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_EINVAL", 2: "NVFP4_EALIGN", 3: "NVFP4_EARCH", 4: "NVFP4_ECUDA",
                  5: "NVFP4_ETIMEOUT"}
@@ -55,8 +56,11 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
     lib.nvfp4_gemm_quant.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, ctypes.POINTER(ColRange), i32,
                                      vp, i64, f32, vp, vp, i64, vp]
+    lib.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.nvfp4_gemm_dynamic.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
-    for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant", "nvfp4_check_fault"):
+    for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
+                 "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_check_fault"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -95,6 +99,11 @@ def nvfp4_quantize(x: int, M: int, K: int, g: float, codes: int, sf: int, stream
     _check(library().nvfp4_quantize(x, M, K, g, codes, sf, stream))
 
 
+def nvfp4_quantize_dynamic(x: int, M: int, K: int, codes: int, sf: int, scale_out: int, workspace: int,
+                           workspace_bytes: int, stream: int) -> None:
+    _check(library().nvfp4_quantize_dynamic(x, M, K, codes, sf, scale_out, workspace, workspace_bytes, stream))
+
+
 def nvfp4_swizzle_sf(sf_linear: int, rows: int, k: int, sf_swizzled: int, stream: int) -> None:
     _check(library().nvfp4_swizzle_sf(sf_linear, rows, k, sf_swizzled, stream))
 
@@ -102,6 +111,11 @@ def nvfp4_swizzle_sf(sf_linear: int, rows: int, k: int, sf_swizzled: int, stream
 def nvfp4_gemm(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha: float, bias: int, y: int,
                stream: int) -> None:
     _check(library().nvfp4_gemm(a, sfa, b, sfb, M, N, K, alpha, bias or None, y, stream))
+
+
+def nvfp4_gemm_dynamic(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_b: float, g_a: int,
+                       bias: int, y: int, stream: int) -> None:
+    _check(library().nvfp4_gemm_dynamic(a, sfa, b, sfb, M, N, K, g_b, g_a, bias or None, y, stream))
 
 
 def nvfp4_gemm_quant(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha: float, bias: int,
@@ -154,12 +168,15 @@ def _need(t, dtype, shape, name):
 @dataclass
 class NVFP4Tensor:
     """A [rows, k] NVFP4 tensor on the GPU: packed codes, swizzled scales and
-    the per-tensor decode scale g."""
+    the per-tensor decode scale g -- a host float, or for a scale measured on
+    the device (quantize_dynamic) ``g = None`` and ``scale`` = the float32
+    device tensor [amax, g]."""
     codes: "object"   # uint8 [rows, k/2]
     sf: "object"      # uint8 [nvfp4_sf_bytes(rows, k)]
-    g: float
+    g: Optional[float]
     rows: int
     k: int
+    scale: "object" = None
 
 
 def calibrate(x, stream=None):
@@ -190,6 +207,26 @@ def quantize(x, g: float, out: Optional[NVFP4Tensor] = None, stream=None) -> NVF
     return out
 
 
+def quantize_dynamic(x, out: Optional[NVFP4Tensor] = None, workspace=None, stream=None) -> NVFP4Tensor:
+    """Quantize bf16 ``x`` [M, K] with the per-tensor scale measured on x in
+    the same launch (g = amax/2688, clamped; nothing is read back).  The
+    result's ``scale`` holds [amax, g] on the device."""
+    torch = _torch()
+    M, K = x.shape
+    _need(x, torch.bfloat16, None, "x")
+    if out is None:
+        out = NVFP4Tensor(torch.empty(M, K // 2, dtype=torch.uint8, device=x.device),
+                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=x.device), None, M, K)
+    if out.scale is None:
+        out.scale = torch.empty(2, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(NVFP4_DYNAMIC_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
+    nvfp4_quantize_dynamic(_ptr(x), M, K, _ptr(out.codes), _ptr(out.sf), _ptr(out.scale), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream))
+    out.g = None
+    return out
+
+
 def swizzle_sf(sf_linear, rows: int, k: int, stream=None):
     """ModelOpt row-major E4M3 scales [rows, k/16] -> swizzled buffer."""
     torch = _torch()
@@ -206,12 +243,17 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = Non
     if a.k != b.k:
         raise ValueError("K mismatch")
     M, N, K = a.rows, b.rows, a.k
-    if alpha is None:
+    if alpha is None and a.g is not None:
         alpha = float(np.float32(a.g) * np.float32(b.g))
     if bias is not None:
         _need(bias, torch.bfloat16, (N,), "bias")
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    if a.g is None and alpha is None:
+        # the activation's scale lives on the device: alpha = fl32(g_a * g_b) in the kernel
+        nvfp4_gemm_dynamic(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(b.g),
+                           _ptr(a.scale) + 4, _ptr(bias), _ptr(y), _stream(stream))
+        return y
     nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias), _ptr(y),
                _stream(stream))
     return y

@@ -203,6 +203,8 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
 
 using namespace nvfp4;
 
+static_assert(kDynamicScratchBytes == NVFP4_DYNAMIC_WORKSPACE_BYTES, "workspace size in the header");
+
 extern "C" {
 
 size_t nvfp4_sf_bytes(int64_t rows, int64_t k) {
@@ -244,6 +246,30 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
   return ok();
 }
 
+nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
+                                    float* scale_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !codes || !sf || !scale_out || !workspace) return fail(NVFP4_EINVAL, "null pointer");
+  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
+  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (workspace_bytes < kDynamicScratchBytes)
+    return fail(NVFP4_EINVAL, "workspace_bytes=%zu is below NVFP4_DYNAMIC_WORKSPACE_BYTES=%zu", workspace_bytes,
+                kDynamicScratchBytes);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0 || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+    return fail(NVFP4_EALIGN, "scale_out and workspace must be 4-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  CUtensorMap tx;
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_quantize_dynamic(tx, x, M, K, codes, sf, scale_out, static_cast<uint32_t*>(workspace),
+                                          static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
+  return ok();
+}
+
 nvfp4_status nvfp4_swizzle_sf(const uint8_t* sf_linear, int64_t rows, int64_t k, uint8_t* sf_swizzled,
                               void* stream) {
   if (!sf_linear || !sf_swizzled) return fail(NVFP4_EINVAL, "null pointer");
@@ -268,6 +294,26 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, 
   const DeviceInfo* dev = nullptr;
   nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev);
   if (st != NVFP4_OK) return st;
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm(maps, p, cg, false, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                                int64_t M, int64_t N, int64_t K, float g_b, const float* g_a, const void* bias,
+                                void* y, void* stream) {
+  if (!y || !g_a) return fail(NVFP4_EINVAL, "null output or scale pointer");
+  if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(g_a) & 3u) != 0) return fail(NVFP4_EALIGN, "g_a must be 4-byte aligned");
+  GemmParams p;
+  GemmTensorMaps maps;
+  GemmConfig cg;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev);
+  if (st != NVFP4_OK) return st;
+  p.alpha_scale = g_a;
   st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
   if (st != NVFP4_OK) return st;
   cudaError_t e = launch_gemm(maps, p, cg, false, static_cast<cudaStream_t>(stream), *dev);

@@ -18,6 +18,7 @@ enum : unsigned {
   kFaultMmaWait = 1u << 1,
   kFaultEpilogueWait = 1u << 2,
   kFaultDrainWait = 1u << 3,
+  kFaultGridWait = 1u << 4,  // a grid-wide barrier did not complete
 };
 
 // Longest a kernel waits on one barrier before giving up (nanoseconds).
@@ -103,6 +104,20 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// Named barrier over `threads` threads of the CTA (a multiple of 32; every
+// warp that takes part arrives with all its threads).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// A 32-bit load with acquire semantics at GPU scope (reads what other CTAs
+// released with fences or atomics).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 

@@ -422,6 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     const int m_padded = (p.M + 127) & ~127;  // rows of the next layer's scale buffer
+    // alpha = g_a * g_b; with a scale measured on the device, g_a is read here
+    const float alpha = p.alpha_scale != nullptr ? __fmul_rn(p.alpha, *p.alpha_scale) : p.alpha;
     for (int tile = cluster; tile < p.num_tiles; tile += num_clusters) {
       const int tm = tile % p.tiles_m;
       const int n0 = (tile / p.tiles_m) * kBN;
@@ -478,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = round_bf16(fmaf(p.alpha, __uint_as_float(r[j]), bias[j]));
+        for (int j = 0; j < 32; ++j) v[j] = round_bf16(fmaf(alpha, __uint_as_float(r[j]), bias[j]));
         if (kFused && act == NVFP4_ACT_GELU_TANH) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = round_bf16(gelu_tanh_f32(v[j]));

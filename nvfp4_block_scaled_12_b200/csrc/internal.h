@@ -29,6 +29,7 @@ struct GemmParams {
   int32_t num_kt;  // k-tiles of 256 elements (last one may be partial)
   int32_t k64;     // K / 64: MMA k-blocks in total, and scale atoms per 128-row block
   float alpha;
+  const float* alpha_scale;   // nullable: if set, the epilogue uses fl(alpha * alpha_scale[0])
   const __nv_bfloat16* bias;  // nullable
   unsigned* fault;
   // operand byte ranges prefetched into L2 at kernel start (A, B, SFA, SFB)
@@ -50,9 +51,22 @@ struct GemmTensorMaps {
   CUtensorMap y;         // bf16 destination of the plain or BF16-range epilogue
 };
 
+// Per-call state of the dynamic-scale quantize.
+struct DynamicScaleArgs {
+  const uint8_t* x;  // bf16 [M, K], for the amax pass
+  uint32_t* scratch; // [0] bits of the grid-wide max |x|, [1] CTAs arrived; both start at zero
+  float* scale_out;  // [0] amax, [1] g, written by CTA 0
+};
+// Bytes of scratch one dynamic-scale quantize uses (zeroed by the launch).
+constexpr size_t kDynamicScratchBytes = 8;
+
 // tmap_x: bf16 [M, K], box 128 rows x 64 columns, 128-byte swizzle.
 cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
                             cudaStream_t stream, const DeviceInfo& dev);
+// Same, with g measured on x in the same (cooperative) launch.
+cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, uint8_t* codes,
+                                    uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream,
+                                    const DeviceInfo& dev);
 cudaError_t launch_calibrate(const void* x, int64_t n, float* out, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out, cudaStream_t stream);
 

@@ -15,6 +15,14 @@
 // previous phase for its next one).  A thread owns one row's 64 elements (four 16-element
 // blocks), so it produces exactly one 4-byte word of the swizzled scale layout
 // and 32 bytes of codes.
+//
+// The dynamic variant measures the per-tensor scale in the same launch: every
+// CTA first takes max |x| over its own tiles (plain 16-byte loads), folds it
+// into a grid-wide maximum and arrives on a grid-wide counter; the producer
+// then starts the TMA ring at once (the tiles do not depend on the scale)
+// while the consumers wait for the counter to reach the grid size, so the
+// second read of a tile usually comes from L2.  The grid is launched
+// cooperatively (every CTA resident), and the wait is bounded.
 #include "internal.h"
 
 namespace nvfp4 {
@@ -30,12 +38,14 @@ constexpr int kQConsumerWarps = 4 * kQGroups;       // 4 quarter-warps per tile
 constexpr int kQThreads = (kQConsumerWarps + 1) * 32;  // + one producer warp
 constexpr uint32_t kQTileBytes = kQRows * kQCols * 2;  // 16 KB of bf16
 constexpr uint32_t kQOffBar = kQStages * kQTileBytes;
-constexpr uint32_t kQSmemBytes = kQOffBar + 2 * kQStages * 8 + 16 + 1024;
+constexpr uint32_t kQOffMax = kQOffBar + 2 * kQStages * 8 + 16;  // per-warp maxima of the amax pass
+constexpr uint32_t kQSmemBytes = kQOffMax + 32 * 4 + 1024;        // + alignment slack
 
+template <bool kDynamic>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t M, int64_t K, float g,
                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int64_t tiles_k, int64_t n_tiles,
-                    unsigned* fault_word) {
+                    unsigned* fault_word, DynamicScaleArgs dyn) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQOffBar);
@@ -53,34 +63,44 @@ __global__ void __launch_bounds__(kQThreads, 1)
   }
   __syncthreads();
   unsigned fault = 0u;
-  // this CTA's tiles are blockIdx.x + j * gridDim.x, j = 0, 1, ...; local
-  // tile j = 4i + g goes to group g, stage g * kQStagesPerGroup + i % 3
+  // This CTA's tiles are blockIdx.x + j * gridDim.x, j = 0 .. my_tiles-1.
+  // The ring carries a sequence of n_seq loads, entry jj = 4i + g going to
+  // consumer group g, stage g * kQStagesPerGroup + i % 3.  The static variant
+  // loads each tile once (entry jj = tile j).  The dynamic one loads them
+  // twice: entries 0 .. my_tiles-1 for the amax pass in order, then the
+  // quantize pass in reverse order, so that its first tiles are the ones
+  // read last (the likeliest to still be in L2).
   const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const int64_t n_seq = kDynamic ? 2 * my_tiles : my_tiles;
+  auto seq_tile = [&](int64_t jj) -> int64_t {
+    const int64_t j = (!kDynamic || jj < my_tiles) ? jj : 2 * my_tiles - 1 - jj;
+    return blockIdx.x + j * gridDim.x;
+  };
 
   if (warp == kQConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
-      int64_t j = 0;
-      for (; j < my_tiles; ++j) {
-        const int64_t i = j / kQGroups;
-        const int stage = static_cast<int>(j % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
+      int64_t jj = 0;
+      for (; jj < n_seq; ++jj) {
+        const int64_t i = jj / kQGroups;
+        const int stage = static_cast<int>(jj % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
         const uint32_t phase = static_cast<uint32_t>((i / kQStagesPerGroup) & 1);
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
           fault = kFaultProducerWait;
           break;
         }
-        const int64_t tile = blockIdx.x + j * gridDim.x;
+        const int64_t tile = seq_tile(jj);
         mbar_arrive_expect_tx(&full[stage], kQTileBytes);
         tma_load_2d(smem + stage * kQTileBytes, &tmap_x, &full[stage], static_cast<int32_t>((tile % tiles_k) * kQCols),
                     static_cast<int32_t>((tile / tiles_k) * kQRows));
       }
       if (fault != 0u) {
         *abort_flag = 1;
-        // let the copies already issued (the last kQStages tiles) land
-        for (int64_t jj = j - 1; jj >= 0 && jj >= j - kQStages; --jj) {
-          const int64_t i = jj / kQGroups;
-          const int stage = static_cast<int>(jj % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
+        // let the copies already issued (the last kQStages entries) land
+        for (int64_t k = jj - 1; k >= 0 && k >= jj - kQStages; --k) {
+          const int64_t i = k / kQGroups;
+          const int stage = static_cast<int>(k % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
           mbar_wait(&full[stage], static_cast<uint32_t>((i / kQStagesPerGroup) & 1), nullptr);
         }
       }
@@ -90,10 +110,59 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int group = warp >> 2;
     const int q = warp & 3;         // rows 32q..32q+31 of each tile
     const int rloc = q * 32 + lane; // this thread's row inside the tile
-    const float d6 = __fmul_rn(6.0f, g);
+    float amax_part = 0.0f;         // dynamic: max |x| over the rows this thread saw
+    bool have_scale = !kDynamic;
+    float d6 = __fmul_rn(6.0f, g);
     const int64_t katoms = K >> 6;
-    for (int64_t j = group; j < my_tiles; j += kQGroups) {
-      const int64_t i = j / kQGroups;
+
+    // Dynamic variant, once per consumer warp (every one of the 16 reaches
+    // it exactly once, so the named barriers below always complete): fold
+    // this CTA's maximum into the grid-wide one, wait (bounded) until every
+    // CTA has, and derive g.
+    auto grid_scale = [&]() {
+      float m = amax_part;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      volatile float* warp_max = reinterpret_cast<volatile float*>(smem + kQOffMax);
+      if (lane == 0) warp_max[warp] = m;
+      named_barrier_sync(1, kQConsumerWarps * 32);
+      if (warp == 0 && lane == 0) {
+        for (int w = 1; w < kQConsumerWarps; ++w) m = fmaxf(m, warp_max[w]);
+        // |x| >= 0, so the float's bit pattern orders like the value
+        atomicMax(dyn.scratch, __float_as_uint(m));
+        __threadfence();
+        atomicAdd(dyn.scratch + 1, 1u);
+        const uint64_t t0 = global_timer_ns();
+        uint32_t arrived;
+        while ((arrived = ld_acquire_gpu(dyn.scratch + 1)) < gridDim.x) {
+          if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) break;
+          __nanosleep(64);
+        }
+        warp_max[kQConsumerWarps] = arrived >= gridDim.x ? __uint_as_float(ld_acquire_gpu(dyn.scratch)) : -1.0f;
+      }
+      named_barrier_sync(1, kQConsumerWarps * 32);
+      const float amax = warp_max[kQConsumerWarps];
+      if (amax < 0.0f) {
+        fault = kFaultGridWait;
+        *abort_flag = 1;
+        return false;
+      }
+      // g = fl(amax / 2688) clamped into [2^-64, 2^64]; 0 for an all-zero tensor
+      g = amax > 0.0f ? fminf(fmaxf(__fdiv_rn(amax, 2688.0f), 0x1p-64f), 0x1p64f) : 0.0f;
+      d6 = __fmul_rn(6.0f, g);
+      if (blockIdx.x == 0 && warp == 0 && lane == 0) {
+        dyn.scale_out[0] = amax;
+        dyn.scale_out[1] = g;
+      }
+      return true;
+    };
+
+    for (int64_t jj = group; jj < n_seq; jj += kQGroups) {
+      if (!have_scale && jj >= my_tiles) {
+        have_scale = true;
+        if (!grid_scale()) break;
+      }
+      const int64_t i = jj / kQGroups;
       const int stage = group * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
       const uint32_t phase = static_cast<uint32_t>((i / kQStagesPerGroup) & 1);
       const bool got = mbar_wait(&full[stage], phase, abort_flag);
@@ -113,7 +182,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);  // this quarter is in registers
 
-      const int64_t tile = blockIdx.x + j * gridDim.x;
+      if (kDynamic && jj < my_tiles) {
+        // amax pass (rows past M arrived zero-filled)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          amax_part = fmaxf(amax_part, fmaxf(fmaxf(fabsf(bf16_lo(v[c].x)), fabsf(bf16_hi(v[c].x))),
+                                             fmaxf(fabsf(bf16_lo(v[c].y)), fabsf(bf16_hi(v[c].y)))));
+          amax_part = fmaxf(amax_part, fmaxf(fmaxf(fabsf(bf16_lo(v[c].z)), fabsf(bf16_hi(v[c].z))),
+                                             fmaxf(fabsf(bf16_lo(v[c].w)), fabsf(bf16_hi(v[c].w)))));
+        }
+        continue;
+      }
+
+      const int64_t tile = seq_tile(jj);
       const int64_t row = (tile / tiles_k) * kQRows + rloc;
       const int64_t katom = tile % tiles_k;  // 64-column group = scale atom column
       uint32_t sfw = 0u;
@@ -133,7 +214,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
           f[8 * h + 6] = bf16_lo(u.w);
           f[8 * h + 7] = bf16_hi(u.w);
         }
-        sfw |= quantize_block16(f, g, d6, cw[2 * b], cw[2 * b + 1]) << (8 * b);
+        if (kDynamic && g == 0.0f) {  // all-zero tensor: zero codes and scales
+          cw[2 * b] = 0u;
+          cw[2 * b + 1] = 0u;
+        } else {
+          sfw |= quantize_block16(f, g, d6, cw[2 * b], cw[2 * b + 1]) << (8 * b);
+        }
       }
       if (row < M) {
         uint8_t* crow = codes + row * (K >> 1) + katom * 32;
@@ -144,6 +230,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       // data was zero-filled by the TMA, so sfw == 0)
       *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 4, katoms)) = sfw;
     }
+    // a group whose entries ended inside the amax pass (or that gave up
+    // there) still takes part in the CTA's scale exchange
+    if (!have_scale) grid_scale();
     if (fault != 0u) *abort_flag = 1;
   }
   if (fault != 0u && lane == 0 && fault_word != nullptr) atomicOr(fault_word, fault);
@@ -182,9 +271,40 @@ cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, flo
   const int64_t tiles_k = (K + kQCols - 1) / kQCols;
   const int64_t n_tiles = tiles_m * tiles_k;
   const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
-  cudaError_t err = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+  cudaError_t err =
+      cudaFuncSetAttribute(quantize_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
   if (err != cudaSuccess) return err;
-  quantize_kernel<<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles, dev.fault);
+  quantize_kernel<false><<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles,
+                                                                   dev.fault, DynamicScaleArgs{});
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, uint8_t* codes,
+                                    uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream,
+                                    const DeviceInfo& dev) {
+  const int64_t tiles_m = (M + kQRows - 1) / kQRows;
+  const int64_t tiles_k = (K + kQCols - 1) / kQCols;
+  const int64_t n_tiles = tiles_m * tiles_k;
+  const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
+  auto kernel = quantize_kernel<true>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+  if (err != cudaSuccess) return err;
+  // the grid-wide maximum and the arrival counter start at zero
+  err = cudaMemsetAsync(scratch, 0, kDynamicScratchBytes, stream);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = kQSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid-wide wait can complete
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const DynamicScaleArgs dyn{static_cast<const uint8_t*>(x), scratch, scale_out};
+  err = cudaLaunchKernelEx(&cfg, kernel, tmap_x, M, K, 0.0f, codes, sf, tiles_k, n_tiles, dev.fault, dyn);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -22,7 +22,8 @@ def declared_functions():
 def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ("nvfp4_sf_bytes", "nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm",
-              "nvfp4_gemm_quant", "nvfp4_check_fault", "nvfp4_last_error"):
+              "nvfp4_gemm_quant", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_check_fault",
+              "nvfp4_last_error"):
         assert n in names
 
 
@@ -84,6 +85,20 @@ def test_gemm_quant_rejects_bad_ranges_on_the_host():
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 256, 0, 1, 64)]))
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([]))
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant, *args([R(0, 64, 0, 1, 0)] * 9))
+
+
+def test_dynamic_entry_points_reject_bad_arguments_on_the_host():
+    W = F.NVFP4_DYNAMIC_WORKSPACE_BYTES
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic, P, 4, 64, P, P, P, 0, W, 0)       # no workspace
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic, P, 4, 64, P, P, P, P, W - 1, 0)   # too small
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic, P, 4, 64, P, P, 0, P, W, 0)       # no scale_out
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic, P, 0, 64, P, P, P, P, W, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic, P, 4, 96, P, P, P, P, W, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_quantize_dynamic, P + 8, 4, 64, P, P, P, P, W, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_quantize_dynamic, P, 4, 64, P, P, P + 2, P, W, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, 1.0, 0, 0, P, 0)   # no g_a
+    _expect(F.NVFP4_EALIGN, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, 1.0, P + 1, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, float("nan"), P, 0, P, 0)
 
 
 def test_calibrate_and_swizzle_reject_bad_arguments_on_the_host():
