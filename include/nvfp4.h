@@ -144,6 +144,32 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K,
                                     void* workspace, size_t workspace_bytes,
                                     void* stream);
 
+/* Bytes of device scratch nvfp4_quantize_dynamic_noalloc holds per device. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+
+/*
+ * nvfp4_quantize_dynamic without a workspace argument.  The source pages have
+ * no counterpart to this entry point: it exists for callers that cannot hand
+ * the library device memory of their own -- e.g. a host program or a plugin
+ * that is given only its input and output buffers and has no device
+ * allocator to draw a workspace from.
+ *   The call allocates nothing.  Its grid state (NVFP4_DYNAMIC_WORKSPACE_BYTES)
+ *   lives in a fixed array in the library's own device memory,
+ *   NVFP4_NOALLOC_SCRATCH_BYTES per device; a call that would need more
+ *   returns EINVAL.  The call zeroes what must start at zero on `stream`
+ *   before the kernel.
+ *   First call on each device: looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current, once; make that first
+ *   call outside any stream capture.
+ *   Calls that overlap in time on the same device (other streams, other host
+ *   threads) share the array and race: order them, e.g. on one stream.
+ * Arguments, results and errors as nvfp4_quantize_dynamic (ECUDA also if the
+ * address lookup fails).
+ */
+nvfp4_status nvfp4_quantize_dynamic_noalloc(const void* x, int64_t M, int64_t K,
+                                            uint8_t* codes, uint8_t* sf, float* scale_out,
+                                            void* stream);
+
 /*
  * Weight preparation: scatter ModelOpt's row-major E4M3 `weight_scale`
  * [rows, k/16] into the swizzled layout the GEMM reads (a byte permutation;

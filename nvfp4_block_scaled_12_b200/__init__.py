@@ -26,6 +26,7 @@ ACT_NONE, ACT_GELU_TANH = 0, 1
 DST_BF16, DST_NVFP4 = 0, 1
 MAX_RANGES = 8
 NVFP4_DYNAMIC_WORKSPACE_BYTES = 8
+NVFP4_NOALLOC_SCRATCH_BYTES = 256
 
 _STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_EINVAL", 2: "NVFP4_EALIGN", 3: "NVFP4_EARCH", 4: "NVFP4_ECUDA",
                  5: "NVFP4_ETIMEOUT"}
@@ -58,9 +59,11 @@ def _load() -> ctypes.CDLL:
                                      vp, i64, f32, vp, vp, i64, vp]
     lib.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.nvfp4_gemm_dynamic.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp, vp]
+    lib.nvfp4_quantize_dynamic_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
-                 "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_check_fault"):
+                 "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
+                 "nvfp4_check_fault"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -102,6 +105,10 @@ def nvfp4_quantize(x: int, M: int, K: int, g: float, codes: int, sf: int, stream
 def nvfp4_quantize_dynamic(x: int, M: int, K: int, codes: int, sf: int, scale_out: int, workspace: int,
                            workspace_bytes: int, stream: int) -> None:
     _check(library().nvfp4_quantize_dynamic(x, M, K, codes, sf, scale_out, workspace, workspace_bytes, stream))
+
+
+def nvfp4_quantize_dynamic_noalloc(x: int, M: int, K: int, codes: int, sf: int, scale_out: int, stream: int) -> None:
+    _check(library().nvfp4_quantize_dynamic_noalloc(x, M, K, codes, sf, scale_out, stream))
 
 
 def nvfp4_swizzle_sf(sf_linear: int, rows: int, k: int, sf_swizzled: int, stream: int) -> None:

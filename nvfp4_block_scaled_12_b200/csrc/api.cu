@@ -77,6 +77,33 @@ nvfp4_status current_device(const DeviceInfo** out) {
   return NVFP4_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch of the no-allocation dynamic quantize.  Callers that cannot hand
+// the library a workspace (a host program or plugin given only its input and
+// output buffers, with no device allocator to draw one from) get the grid
+// state from this fixed array in the library's own device memory instead.
+// One array per device: calls that overlap in time on a device race on it.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = 256;  // the most scratch one call may use
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchBytes / sizeof(uint32_t)];
+uint32_t* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, looked up once per device
+std::mutex g_noalloc_mutex;
+
+// Address of the scratch on device `dev`, which must be current.  The first
+// call per device looks it up (this may load the module on the device, so it
+// belongs outside any stream capture).
+nvfp4_status noalloc_scratch(int dev, uint32_t** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* addr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    g_noalloc_ptr[dev] = static_cast<uint32_t*>(addr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return NVFP4_OK;
+}
+
 // ---------------------------------------------------------------- TMA maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -204,6 +231,7 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
 using namespace nvfp4;
 
 static_assert(kDynamicScratchBytes == NVFP4_DYNAMIC_WORKSPACE_BYTES, "workspace size in the header");
+static_assert(kNoAllocScratchBytes == NVFP4_NOALLOC_SCRATCH_BYTES, "no-allocation scratch size in the header");
 
 extern "C" {
 
@@ -265,6 +293,35 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t
   st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
   cudaError_t e = launch_quantize_dynamic(tx, x, M, K, codes, sf, scale_out, static_cast<uint32_t*>(workspace),
+                                          static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_quantize_dynamic_noalloc(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
+                                            float* scale_out, void* stream) {
+  if (!x || !codes || !sf || !scale_out) return fail(NVFP4_EINVAL, "null pointer");
+  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
+  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0) return fail(NVFP4_EALIGN, "scale_out must be 4-byte aligned");
+  // scratch this call needs (the grid-wide maximum and the arrival counter)
+  const size_t need = kDynamicScratchBytes;
+  if (need > kNoAllocScratchBytes)
+    return fail(NVFP4_EINVAL, "this call needs %zu bytes of scratch; the no-allocation scratch holds %zu", need,
+                kNoAllocScratchBytes);
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  uint32_t* scratch = nullptr;
+  st = noalloc_scratch(dev->device, &scratch);
+  if (st != NVFP4_OK) return st;
+  CUtensorMap tx;
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  if (st != NVFP4_OK) return st;
+  // the launch zeroes the scratch on the stream before the kernel
+  cudaError_t e = launch_quantize_dynamic(tx, x, M, K, codes, sf, scale_out, scratch,
                                           static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
   return ok();
