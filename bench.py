@@ -261,6 +261,90 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- GPU arm
+def extra_workloads(F, torch, synth, device, stream, median_ms, hbm, fp4_peak):
+    """The other measured configurations, one GPU: the FLUX single-stream
+    block pair (fused quantize epilogue vs a bf16 round trip) and the
+    attention-projection token sweep.  Timed like the rest (median, L2
+    flushed before every repetition)."""
+    out = {}
+    # --- single-stream pair: GEMM1 [4608,3072] x [21504,3072]^T whose epilogue
+    # writes Q and GELU(MLP) as NVFP4 (GEMM2's input) and K,V as bf16, then
+    # GEMM2 [4608,15360] x [3072,15360]^T
+    w1l, w2l = synth.SINGLE_IN, synth.SINGLE_OUT
+    M = w1l.m
+    q0, q1 = synth.SINGLE_Q
+    kv0, kv1 = synth.SINGLE_KV
+    m0, m1 = synth.SINGLE_MLP
+    x = w1l.activations().to(device)
+    xq = F.quantize(x, F.global_scale(x))
+    w1 = w1l.weight().to(device)
+    w1q = F.quantize(w1, F.global_scale(w1))
+    w2 = w2l.weight().to(device)
+    w2q = F.quantize(w2, F.global_scale(w2))
+    del w1, w2
+    k2 = w2l.k
+    g2 = 0.05  # the output projection's static input scale
+    a2 = F.NVFP4Tensor(torch.empty(M, k2 // 2, dtype=torch.uint8, device=device),
+                       torch.empty(F.nvfp4_sf_bytes(M, k2), dtype=torch.uint8, device=device), g2, M, k2)
+    y_kv = torch.empty(M, kv1 - kv0, dtype=torch.bfloat16, device=device)
+    y2 = torch.empty(M, w2l.n, dtype=torch.bfloat16, device=device)
+    fused_ranges = [(q0, q1, F.ACT_NONE, F.DST_NVFP4, 0), (kv0, kv1, F.ACT_NONE, F.DST_BF16, 0),
+                    (m0, m1, F.ACT_GELU_TANH, F.DST_NVFP4, q1 - q0)]
+    y_qm = torch.empty(M, k2, dtype=torch.bfloat16, device=device)  # unfused: [Q | GELU(MLP)] in bf16
+    y_all = torch.empty(M, k2 + (kv1 - kv0), dtype=torch.bfloat16, device=device)
+    bf16_ranges = [(q0, q1, F.ACT_NONE, F.DST_BF16, 0), (m0, m1, F.ACT_GELU_TANH, F.DST_BF16, q1 - q0),
+                   (kv0, kv1, F.ACT_NONE, F.DST_BF16, k2)]
+
+    def gemm1_fused():
+        F.gemm_quant(xq, w1q, fused_ranges, y_bf16=y_kv, g_next=g2, next_out=a2, stream=stream)
+
+    def gemm1_bf16():
+        F.gemm_quant(xq, w1q, bf16_ranges, y_bf16=y_all, stream=stream)
+
+    def gemm2():
+        F.gemm(a2, w2q, y=y2, stream=stream)
+
+    def unfused():
+        gemm1_bf16()
+        y_qm.copy_(y_all[:, :k2])  # the quantizer reads rows of K contiguous elements
+        F.quantize(y_qm, g2, out=a2, stream=stream)
+        gemm2()
+
+    f1, f2 = 2 * M * w1l.n * w1l.k, 2 * M * w2l.n * w2l.k
+    t1f = median_ms(gemm1_fused)
+    t1b = median_ms(gemm1_bf16)
+    t2 = median_ms(gemm2)
+    tf = median_ms(lambda: (gemm1_fused(), gemm2()))
+    tu = median_ms(unfused)
+    out["single_stream_pair"] = {
+        "gemm1_fused_ms": t1f, "gemm1_fused_tflops": f1 / (t1f * 1e-3) / 1e12,
+        "gemm1_bf16_out_ms": t1b, "gemm2_ms": t2, "gemm2_tflops": f2 / (t2 * 1e-3) / 1e12,
+        "pair_fused_ms": tf, "pair_unfused_ms": tu,
+        "note": "GEMM1 4608x3072x21504 (Q, GELU(MLP) -> NVFP4 in the epilogue; K,V -> bf16), GEMM2 "
+                "4608x15360x3072; unfused = GEMM1 writing bf16, column copy, quantize, GEMM2"}
+    del y_qm, y_all, y_kv, y2, a2, w1q, w2q, xq, x
+    # --- attention-projection sweep, K = N = 3072
+    sweep = []
+    for wl in synth.SWEEP:
+        x = wl.activations().to(device)
+        g = F.global_scale(x)
+        xq = F.quantize(x, g)
+        w = wl.weight().to(device)
+        wq = F.quantize(w, F.global_scale(w))
+        y = torch.empty(wl.m, wl.n, dtype=torch.bfloat16, device=device)
+        tq = median_ms(lambda: F.quantize(x, g, out=xq, stream=stream))
+        tg = median_ms(lambda: F.gemm(xq, wq, y=y, stream=stream))
+        flops = 2 * wl.m * wl.n * wl.k
+        # min(compute, memory) roofline: A + B + scales in, Y out
+        bytes_ = wl.m * wl.k / 2 + wl.n * wl.k / 2 + (wl.m + wl.n) * wl.k / 16 + wl.m * wl.n * 2
+        t_roof = max(flops / (fp4_peak * 1e12), bytes_ / (hbm * 1e9)) * 1e3
+        sweep.append({"m": wl.m, "quantize_ms": tq, "gemm_ms": tg, "gemm_tflops": flops / (tg * 1e-3) / 1e12,
+                      "frac_of_roofline": t_roof / tg})
+        del x, xq, w, wq, y
+    out["proj_sweep_k3072_n3072"] = sweep
+    return out
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_env()
@@ -397,6 +481,11 @@ def run_ours(args):
 
     ld_ms = median_ms(linear_dynamic)
     F.nvfp4_check_fault()
+    extras = {}
+    if world == 1 and not args.no_extras:
+        hbm_, bf16_, _ = peaks()
+        extras = extra_workloads(F, torch, synth, device, stream, median_ms, hbm_, bf16_ * FP4_PER_BF16)
+        F.nvfp4_check_fault()
 
     if rank == 0:
         hbm, bf16, src = peaks()
@@ -444,6 +533,7 @@ def run_ours(args):
                 "linear_dynamic": {
                     "ms": ld_ms, "tflops": flops / (ld_ms * 1e-3) / 1e12,
                     "note": "MLP-up step with the measured scale: quantize_dynamic + GEMM reading g on the device"},
+                **extras,
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
@@ -467,6 +557,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the single-stream pair and token-sweep measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
