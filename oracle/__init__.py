@@ -13,3 +13,4 @@ from .nvfp4_ref import (  # noqa: F401  (explicit re-exports for readers)
     quantize_dynamic, quantize_nvfp4, round_to_bf16,
     sf_offset, sf_padded_shape, swizzle_sf, tensor_amax, unpack_codes, unswizzle_sf,
 )
+from . import mxfp8_ref  # noqa: F401,E402  (the MXFP8 variant: 32-element blocks, E8M0 scales)
