@@ -37,6 +37,8 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PFLOP/s FP4 vs 2.25 PFLOP/s bf16
 QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
+MX_QUANT_BYTES_PER_ELEM = 2.0 + 1.0 + 1.0 / 32.0  # bf16 in, E4M3 code + E8M0 scale out
+FP8_PER_BF16 = 2.0
 
 
 PROFILES = os.path.join(ROOT, "profiles")
@@ -481,6 +483,13 @@ def run_ours(args):
 
     ld_ms = median_ms(linear_dynamic)
     F.nvfp4_check_fault()
+    # the MXFP8 variant on the same MLP-up shape: E4M3 activations and
+    # weights with one E8M0 scale per 32 elements, no per-tensor scale
+    wq8 = F.quantize_mxfp8(w, stream=stream)
+    xq8 = F.quantize_mxfp8(x, stream=stream)
+    q8_ms = median_ms(lambda: F.quantize_mxfp8(x, out=xq8, stream=stream))
+    g8_ms = median_ms(lambda: F.gemm_mxfp8(xq8, wq8, bias=bias, y=y, stream=stream))
+    F.nvfp4_check_fault()
     extras = {}
     if world == 1 and not args.no_extras:
         hbm_, bf16_, _ = peaks()
@@ -533,6 +542,14 @@ def run_ours(args):
                 "linear_dynamic": {
                     "ms": ld_ms, "tflops": flops / (ld_ms * 1e-3) / 1e12,
                     "note": "MLP-up step with the measured scale: quantize_dynamic + GEMM reading g on the device"},
+                "mxfp8": {
+                    "quantize_ms": q8_ms,
+                    "quantize_gbs": M * K * MX_QUANT_BYTES_PER_ELEM / (q8_ms * 1e-3) / 1e9,
+                    "quantize_frac_of_hbm": M * K * MX_QUANT_BYTES_PER_ELEM / (q8_ms * 1e-3) / 1e9 / hbm,
+                    "gemm_ms": g8_ms, "gemm_tflops": flops / (g8_ms * 1e-3) / 1e12,
+                    "gemm_frac_of_fp8_peak": flops / (g8_ms * 1e-3) / 1e12 / (bf16 * FP8_PER_BF16),
+                    "note": "MLP-up shape with MXFP8 operands (E4M3, E8M0 per 32); quantize bytes 2 + 1 + 1/32 "
+                            "per element; FP8 peak = measured bf16 burst x 2 (nominal FP8/bf16 dense ratio)"},
                 **extras,
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

@@ -254,6 +254,56 @@ nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_
                               int64_t k_next, void* stream);
 
 /*
+ * ------------------------------------------------------------------------
+ * MXFP8 variant ("NVIDIA FP4 format" news page, paragraph 1: 8-bit E4M3/E5M2
+ * elements in 32-element blocks, Open Compute Project microscaling; the
+ * page's 1.26x end-to-end figure for MXFP8 next to NVFP4's 1.68x).  E4M3
+ * elements, one E8M0 scale (a power of two, 2^(byte - 127)) per 32 elements
+ * along K, no per-tensor scale.
+ *   codes   [rows, K] uint8, one E4M3 byte per element
+ *   scales  nvfp4_mxfp8_sf_bytes(rows, K) bytes: the same 512-byte atom
+ *           layout as the NVFP4 scales, with one scale column per 32
+ *           elements (K/32 columns padded to a multiple of 4; padding 0)
+ * ------------------------------------------------------------------------
+ */
+
+/* Size of the swizzled MXFP8 scale buffer: ceil(rows/128)*128 *
+ * ceil(k/128)*4.  0 if rows < 1 or k < 32 or k % 32 != 0.  Host-only. */
+size_t nvfp4_mxfp8_sf_bytes(int64_t rows, int64_t k);
+
+/*
+ * bf16 -> MXFP8.  For each row and each 32-element block along K:
+ *     amax = max |x_i|
+ *     amax == 0:  scale byte 0;  codes E4M3(x_i) (zeros, sign kept)
+ *     else        s = clamp(floor(log2 amax) - 8, -127, 127);  scale byte s + 127
+ *                 code_i = E4M3_satfinite(fl(x_i * 2^-s))   (RNE, +-448)
+ * (the microscaling conversion: 8 is the exponent of E4M3's largest normal,
+ * 448 = 1.75 * 2^8, so the block maximum lands in [256, 448]).
+ *   x      [M, K] bf16, finite
+ *   codes  [M, K] uint8, written;  sf  nvfp4_mxfp8_sf_bytes(M, K), written
+ *          including its zero padding.
+ * M >= 1, K % 64 == 0.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_mxfp8_quantize(const void* x, int64_t M, int64_t K,
+                                  uint8_t* codes, uint8_t* sf, void* stream);
+
+/*
+ * Block-scaled MXFP8 GEMM on the tensor cores (tcgen05, kind::mxf8f6f4, one
+ * E8M0 scale per 32 elements), dequant folded into the epilogue:
+ *     y[m, n] = bf16_rn( alpha * sum_k a_hat[m,k] * b_hat[n,k] + bias[n] )
+ * with a_hat = e4m3(a) * 2^(sfa - 127), b_hat likewise.
+ *   a  [M, K] codes, sfa nvfp4_mxfp8_sf_bytes(M, K);  b [N, K] codes (the
+ *   weight, PyTorch [out, in]), sfb nvfp4_mxfp8_sf_bytes(N, K);
+ *   alpha finite (1 for a plain MXFP8 layer);  bias [N] bf16 or NULL;
+ *   y [M, N] bf16, written.
+ * M >= 1, N >= 8 with N % 8 == 0, K % 64 == 0.  Errors: EINVAL, EALIGN,
+ * EARCH, ECUDA; a barrier time-out records NVFP4_ETIMEOUT (nvfp4_check_fault).
+ */
+nvfp4_status nvfp4_mxfp8_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                              const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                              float alpha, const void* bias, void* y, void* stream);
+
+/*
  * Synchronize the current device, then read and clear its fault word.
  * Returns NVFP4_ETIMEOUT if any kernel of this library gave up on a barrier
  * wait since the last check, NVFP4_ECUDA if the synchronize failed, else

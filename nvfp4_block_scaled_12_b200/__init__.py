@@ -60,10 +60,14 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.nvfp4_gemm_dynamic.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp, vp]
     lib.nvfp4_quantize_dynamic_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+    lib.nvfp4_mxfp8_sf_bytes.argtypes = [i64, i64]
+    lib.nvfp4_mxfp8_sf_bytes.restype = ctypes.c_size_t
+    lib.nvfp4_mxfp8_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+    lib.nvfp4_mxfp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
-                 "nvfp4_check_fault"):
+                 "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_check_fault"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -131,6 +135,19 @@ def nvfp4_gemm_quant(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int,
     arr = (ColRange * len(ranges))(*ranges)
     _check(library().nvfp4_gemm_quant(a, sfa, b, sfb, M, N, K, alpha, bias or None, arr, len(ranges), y_bf16 or None,
                                  ldy, g_next, codes_next or None, sf_next or None, k_next, stream))
+
+
+def nvfp4_mxfp8_sf_bytes(rows: int, k: int) -> int:
+    return int(library().nvfp4_mxfp8_sf_bytes(rows, k))
+
+
+def nvfp4_mxfp8_quantize(x: int, M: int, K: int, codes: int, sf: int, stream: int) -> None:
+    _check(library().nvfp4_mxfp8_quantize(x, M, K, codes, sf, stream))
+
+
+def nvfp4_mxfp8_gemm(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha: float, bias: int, y: int,
+                     stream: int) -> None:
+    _check(library().nvfp4_mxfp8_gemm(a, sfa, b, sfb, M, N, K, alpha, bias or None, y, stream))
 
 
 def nvfp4_check_fault() -> None:
@@ -232,6 +249,43 @@ def quantize_dynamic(x, out: Optional[NVFP4Tensor] = None, workspace=None, strea
                            workspace.numel() * workspace.element_size(), _stream(stream))
     out.g = None
     return out
+
+
+@dataclass
+class MXFP8Tensor:
+    """A [rows, k] MXFP8 tensor on the GPU: E4M3 codes (one byte per element)
+    and swizzled E8M0 scales (one per 32 elements)."""
+    codes: "object"   # uint8 [rows, k]
+    sf: "object"      # uint8 [nvfp4_mxfp8_sf_bytes(rows, k)]
+    rows: int
+    k: int
+
+
+def quantize_mxfp8(x, out: Optional[MXFP8Tensor] = None, stream=None) -> MXFP8Tensor:
+    """Quantize bf16 ``x`` [M, K] to MXFP8 (power-of-two block scales)."""
+    torch = _torch()
+    M, K = x.shape
+    _need(x, torch.bfloat16, None, "x")
+    if out is None:
+        out = MXFP8Tensor(torch.empty(M, K, dtype=torch.uint8, device=x.device),
+                          torch.empty(nvfp4_mxfp8_sf_bytes(M, K), dtype=torch.uint8, device=x.device), M, K)
+    nvfp4_mxfp8_quantize(_ptr(x), M, K, _ptr(out.codes), _ptr(out.sf), _stream(stream))
+    return out
+
+
+def gemm_mxfp8(a: MXFP8Tensor, b: MXFP8Tensor, bias=None, alpha: float = 1.0, y=None, stream=None):
+    """y = bf16(alpha * a_hat @ b_hat^T + bias) for MXFP8 operands."""
+    torch = _torch()
+    if a.k != b.k:
+        raise ValueError("K mismatch")
+    M, N, K = a.rows, b.rows, a.k
+    if bias is not None:
+        _need(bias, torch.bfloat16, (N,), "bias")
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    nvfp4_mxfp8_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias),
+                     _ptr(y), _stream(stream))
+    return y
 
 
 def swizzle_sf(sf_linear, rows: int, k: int, stream=None):

@@ -155,11 +155,13 @@ nvfp4_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base,
 // Swizzled scale buffer of a [rows, k] tensor seen as [row blocks][k/64
 // atoms][128 x u32]; the box covers 4 atoms (one 256-wide k-tile) of
 // `box_blocks` row blocks.  Out-of-range atoms and blocks read as zero.
-nvfp4_status make_sf_tmap(CUtensorMap* m, const void* sf, int64_t rows, int64_t k, uint32_t box_blocks,
-                          const char* what) {
-  const uint64_t dims[3] = {128, static_cast<uint64_t>(k / 64), static_cast<uint64_t>((rows + 127) / 128)};
-  const uint64_t strides[2] = {512, static_cast<uint64_t>(k / 64) * 512};
-  const uint32_t box[3] = {128, 4, box_blocks};
+// Swizzled scales as [row blocks][atoms][128 x u32]; one box = box_atoms
+// atoms of box_blocks row blocks.
+nvfp4_status make_sf_tmap(CUtensorMap* m, const void* sf, int64_t rows, int64_t atoms, uint32_t box_atoms,
+                          uint32_t box_blocks, const char* what) {
+  const uint64_t dims[3] = {128, static_cast<uint64_t>(atoms), static_cast<uint64_t>((rows + 127) / 128)};
+  const uint64_t strides[2] = {512, static_cast<uint64_t>(atoms) * 512};
+  const uint32_t box[3] = {128, box_atoms, box_blocks};
   return make_tmap_nd(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, sf, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
                       what);
 }
@@ -170,9 +172,10 @@ bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
 
 // Checks shared by the two GEMM entry points; fills the operand part of p
 // and the operand tensor maps.
+// mx: MXFP8 operands (one E4M3 byte per element, E8M0 scales per 32).
 nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
                          int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, GemmTensorMaps* maps,
-                         GemmConfig* cfg, const DeviceInfo** dev) {
+                         GemmConfig* cfg, const DeviceInfo** dev, bool mx = false) {
   if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
   if (M < 1 || M > INT32_MAX / 2) return fail(NVFP4_EINVAL, "M=%lld out of range", (long long)M);
   if (N < 8 || N % 8 != 0 || N > INT32_MAX / 2)
@@ -197,32 +200,37 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   const int64_t tiles = static_cast<int64_t>(p->tiles_m) * p->tiles_n;
   if (tiles > INT32_MAX) return fail(NVFP4_EINVAL, "problem too large");
   p->num_tiles = static_cast<int32_t>(tiles);
-  p->num_kt = static_cast<int32_t>((K + 255) / 256);
-  p->k64 = static_cast<int32_t>(K / 64);
+  // a k-tile is 128 bytes of every operand row: 256 fp4 or 128 fp8 elements
+  const int64_t row_bytes = mx ? K : K / 2;
+  p->num_kt = static_cast<int32_t>((row_bytes + 127) / 128);
+  p->kblocks = static_cast<int32_t>(mx ? K / 32 : K / 64);
   p->alpha = alpha;
   p->bias = static_cast<const __nv_bfloat16*>(bias);
   p->fault = (*dev)->fault;
   p->pf_ptr[0] = b;  // weights first: every tile of a wave touches new weight rows
-  p->pf_bytes[0] = static_cast<uint64_t>(N) * static_cast<uint64_t>(K / 2);
+  p->pf_bytes[0] = static_cast<uint64_t>(N) * static_cast<uint64_t>(row_bytes);
   p->pf_ptr[1] = a;
-  p->pf_bytes[1] = static_cast<uint64_t>(M) * static_cast<uint64_t>(K / 2);
+  p->pf_bytes[1] = static_cast<uint64_t>(M) * static_cast<uint64_t>(row_bytes);
   p->pf_ptr[2] = sfb;
-  p->pf_bytes[2] = nvfp4_sf_bytes(N, K);
+  p->pf_bytes[2] = mx ? nvfp4_mxfp8_sf_bytes(N, K) : nvfp4_sf_bytes(N, K);
   p->pf_ptr[3] = sfa;
-  p->pf_bytes[3] = nvfp4_sf_bytes(M, K);
+  p->pf_bytes[3] = mx ? nvfp4_mxfp8_sf_bytes(M, K) : nvfp4_sf_bytes(M, K);
 
-  st = make_tmap(&maps->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B,
-                 "A");
+  st = make_tmap(&maps->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, row_bytes, M, row_bytes, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B, "A");
   if (st != NVFP4_OK) return st;
-  st = make_tmap(&maps->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K / 2, N, K / 2, 128, bn / cg,
+  st = make_tmap(&maps->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, row_bytes, N, row_bytes, 128, bn / cg,
                  CU_TENSOR_MAP_SWIZZLE_128B, "B");
   if (st != NVFP4_OK) return st;
-  st = make_sf_tmap(&maps->sfa, sfa, M, K, 1, "A scales");
+  // scale atoms per 128-row block, and atoms per k-tile
+  const int64_t atoms = mx ? (K / 32 + 3) / 4 : K / 64;
+  const uint32_t box_atoms = mx ? 1u : 4u;
+  st = make_sf_tmap(&maps->sfa, sfa, M, atoms, box_atoms, 1, "A scales");
   if (st != NVFP4_OK) return st;
   // 128-row scale blocks one B tile can touch: a width that is not a
   // multiple of 128 may start in the middle of a block
   const uint32_t sfb_blocks = static_cast<uint32_t>(bn % 128 == 0 ? bn / 128 : bn / 128 + 1);
-  return make_sf_tmap(&maps->sfb, sfb, N, K, sfb_blocks, "B scales");
+  return make_sf_tmap(&maps->sfb, sfb, N, atoms, box_atoms, sfb_blocks, "B scales");
 }
 
 }  // namespace
@@ -234,6 +242,47 @@ static_assert(kDynamicScratchBytes == NVFP4_DYNAMIC_WORKSPACE_BYTES, "workspace 
 static_assert(kNoAllocScratchBytes == NVFP4_NOALLOC_SCRATCH_BYTES, "no-allocation scratch size in the header");
 
 extern "C" {
+
+size_t nvfp4_mxfp8_sf_bytes(int64_t rows, int64_t k) {
+  if (rows < 1 || k < 32 || k % 32 != 0) return 0;
+  const int64_t rp = (rows + 127) / 128 * 128;
+  const int64_t cp = (k / 32 + 3) / 4 * 4;
+  return static_cast<size_t>(rp) * static_cast<size_t>(cp);
+}
+
+nvfp4_status nvfp4_mxfp8_quantize(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf, void* stream) {
+  if (!x || !codes || !sf) return fail(NVFP4_EINVAL, "null pointer");
+  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
+  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  CUtensorMap tx;
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_quantize_mxfp8(tx, M, K, codes, sf, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "mxfp8 quantize launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_mxfp8_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
+                              int64_t N, int64_t K, float alpha, const void* bias, void* y, void* stream) {
+  if (!y) return fail(NVFP4_EINVAL, "null output pointer");
+  if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
+  GemmParams p;
+  GemmTensorMaps maps;
+  GemmConfig cg;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev, true);
+  if (st != NVFP4_OK) return st;
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm(maps, p, cg, false, true, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "mxfp8 gemm launch");
+  return ok();
+}
 
 size_t nvfp4_sf_bytes(int64_t rows, int64_t k) {
   if (rows < 1 || k < 16 || k % 16 != 0) return 0;
@@ -353,7 +402,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, 
   if (st != NVFP4_OK) return st;
   st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_gemm(maps, p, cg, false, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_gemm(maps, p, cg, false, false, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return ok();
 }
@@ -373,7 +422,7 @@ nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint
   p.alpha_scale = g_a;
   st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_gemm(maps, p, cg, false, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_gemm(maps, p, cg, false, false, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return ok();
 }
@@ -446,7 +495,7 @@ nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_
   p.codes_next = codes_next;
   p.sf_next = sf_next;
   p.k_next = static_cast<int32_t>(k_next);
-  cudaError_t e = launch_gemm(maps, p, cg, true, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_gemm(maps, p, cg, true, false, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_quant launch");
   return ok();
 }

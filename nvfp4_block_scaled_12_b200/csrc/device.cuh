@@ -83,6 +83,37 @@ __device__ __forceinline__ uint32_t quantize_block16(const float (&v)[16], float
   return s;
 }
 
+// MXFP8 block (OCP microscaling): 32 fp32 values (exactly representable in
+// bf16) -> 32 E4M3 bytes in 8 little-endian words and the E8M0 scale byte.
+//   amax == 0: scale byte 0 (2^-127);  else s = clamp(floor(log2 amax) - 8,
+//   -127, 127), scale byte s + 127;  code_i = E4M3_satfinite(fl(v_i * 2^-s)).
+__device__ __forceinline__ uint32_t quantize_mx_block32(const float (&v)[32], uint32_t (&w)[8]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t bits = __float_as_uint(amax);
+  int e;  // floor(log2(amax)) for amax > 0
+  if (bits >= 0x00800000u)
+    e = static_cast<int>(bits >> 23) - 127;
+  else
+    e = (31 - __clz(static_cast<int>(bits))) - 149;  // fp32 subnormal: bits * 2^-149
+  int s = bits == 0u ? -127 : e - 8;
+  s = s < -127 ? -127 : (s > 127 ? 127 : s);
+  // 2^-s exactly: a normal float for s <= 126, the subnormal 2^-127 for s = 127
+  const float inv = s <= 126 ? __uint_as_float(static_cast<uint32_t>(127 - s) << 23) : __uint_as_float(0x00400000u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint16_t lo, hi;
+    // cvt puts its first source in the high byte: pass (odd, even)
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(__fmul_rn(v[4 * i + 1], inv)),
+        "f"(__fmul_rn(v[4 * i + 0], inv)));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(__fmul_rn(v[4 * i + 3], inv)),
+        "f"(__fmul_rn(v[4 * i + 2], inv)));
+    w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  }
+  return static_cast<uint32_t>(s + 127);
+}
+
 // Byte offset of logical scale (row r, scale column c) in the swizzled
 // scale-factor buffer with `katoms` 4-column atoms per 128-row block.
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t katoms) {
@@ -406,6 +437,41 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
          | (1u << 10)                               // B format: E2M1
          | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16 (scale format bit 23 = 0: UE4M3)
+}
+
+// Instruction descriptor of the MXFP8 block-scaled MMA: E4M3 x E4M3 -> fp32,
+// both operands K-major, UE8M0 scales, dense K = 32.  One 32-bit TMEM scale
+// word holds the scales of four consecutive 32-element blocks; sf_id picks the
+// byte this MMA uses, for A (bits 29-30) and B (bits 4-5).
+__host__ __device__ constexpr uint32_t idesc_mxf8(int m, int n, uint32_t sf_id) {
+  return (sf_id << 4)                               // B scale byte
+         | (0u << 7)                                // A format: E4M3
+         | (0u << 10)                               // B format: E4M3
+         | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
+         | (1u << 23)                               // scale format: UE8M0
+         | (static_cast<uint32_t>(m >> 4) << 24)    // M / 16
+         | (sf_id << 29);                           // A scale byte
+}
+
+// MXFP8 MMA (kind::mxf8f6f4, one E8M0 scale per 32 elements); the scale
+// addresses carry the scale byte in their top two bits, as the descriptor does.
+__device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
 }
 
 // Registers -> TMEM: 32 lanes (this warp's quarter) x 4 / 8 consecutive

@@ -46,22 +46,27 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kBKBytes = 128;   // 256 fp4 elements per row per stage
+constexpr int kBKBytes = 128;   // per row per stage: 256 fp4 or 128 fp8 elements
 constexpr uint32_t kABytes = 128 * kBKBytes;  // 16 KB: this CTA's 128 rows of A
-constexpr uint32_t kSfaBytes = 4 * 512;       // 4 k-blocks x one 128-row atom
 constexpr int kThreads = 352;
 constexpr int kProducers = 2;  // warps 0 and 10
 constexpr uint32_t kTmemCols = 512;
 
-// kCG: CTAs per tile; kBN: tile width; kAcc: accumulator buffers in TMEM.
-template <int kCG, int kBN, int kAcc>
+// kCG: CTAs per tile; kBN: tile width; kAcc: accumulator buffers in TMEM;
+// kMx: MXFP8 operands (E4M3, one E8M0 scale per 32 elements) instead of NVFP4.
+template <int kCG, int kBN, int kAcc, bool kMx>
 struct Cfg {
+  // 512-byte scale atoms (128 rows x 4 scale columns) per 128-row block and
+  // k-tile: NVFP4's k-tile is 4 MMA k-blocks of 64 elements with one 4-scale
+  // word per row each; MXFP8's is 4 k-blocks of 32 whose scales share one word.
+  static constexpr int kAtoms = kMx ? 1 : 4;
+  static constexpr uint32_t kSfaBytes = kAtoms * 512;
   static constexpr int kBNc = kBN / kCG;  // B rows per CTA
   static constexpr uint32_t kBBytes = kBNc * kBKBytes;
   static constexpr int kChunks = kBN / 32;
   // 128-row scale blocks a B tile can touch (a 192-wide tile may start mid-block)
   static constexpr int kSfbBlocks = kBN % 128 == 0 ? kBN / 128 : kBN / 128 + 1;
-  static constexpr uint32_t kSfbBytes = kSfbBlocks * 4 * 512;
+  static constexpr uint32_t kSfbBytes = kSfbBlocks * kAtoms * 512;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStagesFit = (224 * 1024 - 4 * 2 * 2048) / kStageBytes;
   // a multiple of the producer count: each stage then has a single producer
@@ -73,11 +78,12 @@ struct Cfg {
   // j - kSfSlots has arrived on that k-tile's empty barrier, which can only
   // be the phase they wait for while kSfSlots <= kStages.
   static constexpr uint32_t kSfbGroups = kBN / 32;       // 32-row groups of B scales per k-block
-  static constexpr uint32_t kSfbSlotCols = 4 * kSfbGroups;
-  static constexpr int kSfSlotsFit = (kTmemCols - kAcc * kBN) / (16 + kSfbSlotCols);
+  static constexpr uint32_t kSfaSlotCols = kMx ? 4 : 16;
+  static constexpr uint32_t kSfbSlotCols = kMx ? (kSfbGroups + 7) / 8 * 8 : 4 * kSfbGroups;
+  static constexpr int kSfSlotsFit = (kTmemCols - kAcc * kBN) / (kSfaSlotCols + kSfbSlotCols);
   static constexpr int kSfSlots = kSfSlotsFit < kStages ? (kSfSlotsFit > 8 ? 8 : kSfSlotsFit) : kStages;
   static constexpr uint32_t kSfaCol = kAcc * kBN;
-  static constexpr uint32_t kSfbCol = kSfaCol + 16 * kSfSlots;
+  static constexpr uint32_t kSfbCol = (kSfaCol + kSfaSlotCols * kSfSlots + 7) / 8 * 8;
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
   static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
@@ -92,7 +98,7 @@ struct Cfg {
   static_assert(kBN % 32 == 0 && kBN / kCG % 8 == 0, "tile width");
   static_assert(kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
   static_assert(kSfSlots >= 2 && kSfSlots <= kStages, "TMEM budget");
-  static_assert(kSfaCol % 16 == 0 && kSfbCol % 8 == 0 && kSfbSlotCols % 8 == 0, "tcgen05.st column alignment");
+  static_assert(kSfaCol % kSfaSlotCols == 0 && kSfbCol % 8 == 0 && kSfbSlotCols % 8 == 0, "tcgen05.st column alignment");
   static_assert(kSfbCol + kSfSlots * kSfbSlotCols <= kTmemCols, "TMEM budget");
   static_assert(kStages >= 3, "pipeline depth");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -126,12 +132,13 @@ __device__ __forceinline__ void store_chunk_bf16(const CUtensorMap* tmap, uint8_
   }
 }
 
-template <int kCG, int kBN, int kAcc, bool kFused>
+template <int kCG, int kBN, int kAcc, bool kFused, bool kMx>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ GemmParams p) {
-  using C = Cfg<kCG, kBN, kAcc>;
+  using C = Cfg<kCG, kBN, kAcc, kMx>;
+  static_assert(!(kFused && kMx), "the fused quantize epilogue writes NVFP4 after an NVFP4 GEMM");
   constexpr int S = C::kStages;
   constexpr int R = C::kSfSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n0 = (tile / p.tiles_m) * kBN;
         const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
         if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
-        mbar_arrive_expect_tx(&sfin[stage], kSfaBytes + C::kSfbBytes);
+        mbar_arrive_expect_tx(&sfin[stage], C::kSfaBytes + C::kSfbBytes);
         uint8_t* sa = smem + C::kOffA + stage * kABytes;
         uint8_t* sb = smem + C::kOffB + stage * C::kBBytes;
         if (kCG == 2) {
@@ -247,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sa, &tmap_a, &full[stage], kt * kBKBytes, row_block * 128);
           tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
         }
-        tma_load_3d(smem + C::kOffSfa + stage * kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * 4, row_block);
-        tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * 4, n0 >> 7);
+        tma_load_3d(smem + C::kOffSfa + stage * C::kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * C::kAtoms, row_block);
+        tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * C::kAtoms, n0 >> 7);
       }
       if (fault != 0u) {
         *abort_flag = 1;
@@ -264,7 +271,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (group leader)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_nvf4(128 * kCG, kBN);
+      // one MMA k-block: NVFP4 reads 4 scale columns per k-block; MXFP8 reads
+      // byte kb of the k-tile's scale words (named in the descriptor and in
+      // the top two bits of the scale addresses)
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb, int kb, uint32_t accum) {
+        if constexpr (kMx) {
+          const uint32_t idesc = idesc_mxf8(128 * kCG, kBN, static_cast<uint32_t>(kb));
+          const uint32_t sel = static_cast<uint32_t>(kb) << 30;
+          if (kCG == 2)
+            tc_mma_mxf8_pair(d, ad, bd, idesc, sfa | sel, sfb | sel, accum);
+          else
+            tc_mma_mxf8(d, ad, bd, idesc, sfa | sel, sfb | sel, accum);
+        } else {
+          constexpr uint32_t idesc = idesc_nvf4(128 * kCG, kBN);
+          if (kCG == 2)
+            tc_mma_nvf4_pair(d, ad, bd, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
+          else
+            tc_mma_nvf4(d, ad, bd, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
+        }
+      };
       int stage = 0;
       uint32_t phase = 0;
       int slot = 0;
@@ -283,10 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const int nkb = min(4, p.k64 - kt * 4);
+          const int nkb = min(4, p.kblocks - kt * 4);
           const uint32_t sa = smem_u32(smem + C::kOffA + stage * kABytes);
           const uint32_t sb = smem_u32(smem + C::kOffB + stage * C::kBBytes);
-          const uint32_t sfa = tmem_base + C::kSfaCol + static_cast<uint32_t>(slot) * 16u;
+          const uint32_t sfa = tmem_base + C::kSfaCol + static_cast<uint32_t>(slot) * C::kSfaSlotCols;
           const uint32_t sfb = tmem_base + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols;
           // One thread issues the MMAs and the tensor pipe queues few of them,
           // so the instructions between two MMAs are on the critical path: the
@@ -296,25 +321,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = sdesc_kmajor_sw128(sa), bd = sdesc_kmajor_sw128(sb);
           if (nkb == 4) {
             const uint32_t first = kt != 0 ? 1u : 0u;
-            if (kCG == 2) {
-              tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, sfa, sfb, first);
-              tc_mma_nvf4_pair(d_tmem, ad + 2, bd + 2, idesc, sfa + 4, sfb + C::kSfbGroups, 1u);
-              tc_mma_nvf4_pair(d_tmem, ad + 4, bd + 4, idesc, sfa + 8, sfb + 2 * C::kSfbGroups, 1u);
-              tc_mma_nvf4_pair(d_tmem, ad + 6, bd + 6, idesc, sfa + 12, sfb + 3 * C::kSfbGroups, 1u);
-            } else {
-              tc_mma_nvf4(d_tmem, ad, bd, idesc, sfa, sfb, first);
-              tc_mma_nvf4(d_tmem, ad + 2, bd + 2, idesc, sfa + 4, sfb + C::kSfbGroups, 1u);
-              tc_mma_nvf4(d_tmem, ad + 4, bd + 4, idesc, sfa + 8, sfb + 2 * C::kSfbGroups, 1u);
-              tc_mma_nvf4(d_tmem, ad + 6, bd + 6, idesc, sfa + 12, sfb + 3 * C::kSfbGroups, 1u);
-            }
+            mma(d_tmem, ad, bd, sfa, sfb, 0, first);
+            mma(d_tmem, ad + 2, bd + 2, sfa, sfb, 1, 1u);
+            mma(d_tmem, ad + 4, bd + 4, sfa, sfb, 2, 1u);
+            mma(d_tmem, ad + 6, bd + 6, sfa, sfb, 3, 1u);
           } else {
-            for (int kb = 0; kb < nkb; ++kb) {
-              const uint32_t accum = (kt | kb) != 0 ? 1u : 0u;
-              if (kCG == 2)
-                tc_mma_nvf4_pair(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
-              else
-                tc_mma_nvf4(d_tmem, ad + 2 * kb, bd + 2 * kb, idesc, sfa + kb * 4, sfb + kb * C::kSfbGroups, accum);
-            }
+            for (int kb = 0; kb < nkb; ++kb) mma(d_tmem, ad + 2 * kb, bd + 2 * kb, sfa, sfb, kb, (kt | kb) != 0 ? 1u : 0u);
           }
           // frees the smem stage and the scale slot once these MMAs have read them
           commit_group(&empty[stage]);
@@ -370,38 +382,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // All loads first (atoms past K arrived zero-filled), then a few wide
         // stores: a shared load is not reordered across a tcgen05.st.
-        const uint8_t* ssfa = smem + C::kOffSfa + stage * kSfaBytes + lane * 16;
+        const uint8_t* ssfa = smem + C::kOffSfa + stage * C::kSfaBytes + lane * 16;
         const uint8_t* ssfb = smem + C::kOffSfb + stage * C::kSfbBytes + lane * 16;
-        uint32_t sa[16];
-        uint32_t sb[4 * C::kSfbGroups];
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512);
-          sa[4 * kb + 0] = v.x;
-          sa[4 * kb + 1] = v.y;
-          sa[4 * kb + 2] = v.z;
-          sa[4 * kb + 3] = v.w;
+        if constexpr (kMx) {
+          // one atom per 128-row block: word j of lane l's chunk = the four
+          // 32-element-block scales of row 32j + l
+          const uint4 a = *reinterpret_cast<const uint4*>(ssfa);
           uint32_t w[4 * C::kSfbBlocks];
 #pragma unroll
           for (int blk = 0; blk < C::kSfbBlocks; ++blk) {
-            const uint4 u = *reinterpret_cast<const uint4*>(ssfb + blk * 4 * 512 + kb * 512);
+            const uint4 u = *reinterpret_cast<const uint4*>(ssfb + blk * 512);
             w[4 * blk + 0] = u.x;
             w[4 * blk + 1] = u.y;
             w[4 * blk + 2] = u.z;
             w[4 * blk + 3] = u.w;
           }
+          uint32_t sb[C::kSfbSlotCols];
 #pragma unroll
-          for (int g = 0; g < static_cast<int>(C::kSfbGroups); ++g) {
-            if constexpr (kBN % 128 != 0)
-              sb[kb * C::kSfbGroups + g] = mid ? w[g + 2] : w[g];
+          for (int g = 0; g < static_cast<int>(C::kSfbSlotCols); ++g) {
+            if (g >= static_cast<int>(C::kSfbGroups))
+              sb[g] = 0u;
+            else if constexpr (kBN % 128 != 0)
+              sb[g] = mid ? w[g + 2] : w[g];
             else
-              sb[kb * C::kSfbGroups + g] = w[g];
+              sb[g] = w[g];
           }
-        }
-        tmem_st_32x32b_x16(t_quarter + C::kSfaCol + static_cast<uint32_t>(slot) * 16u, sa);
+          tmem_st_32x32b_x4(t_quarter + C::kSfaCol + static_cast<uint32_t>(slot) * C::kSfaSlotCols, a);
 #pragma unroll
-        for (int c = 0; c < static_cast<int>(C::kSfbSlotCols / 8); ++c)
-          tmem_st_32x32b_x8(t_quarter + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols + c * 8, sb + 8 * c);
+          for (int c = 0; c < static_cast<int>(C::kSfbSlotCols / 8); ++c)
+            tmem_st_32x32b_x8(t_quarter + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols + c * 8,
+                              sb + 8 * c);
+        } else {
+          uint32_t sa[16];
+          uint32_t sb[4 * C::kSfbGroups];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512);
+            sa[4 * kb + 0] = v.x;
+            sa[4 * kb + 1] = v.y;
+            sa[4 * kb + 2] = v.z;
+            sa[4 * kb + 3] = v.w;
+            uint32_t w[4 * C::kSfbBlocks];
+#pragma unroll
+            for (int blk = 0; blk < C::kSfbBlocks; ++blk) {
+              const uint4 u = *reinterpret_cast<const uint4*>(ssfb + blk * 4 * 512 + kb * 512);
+              w[4 * blk + 0] = u.x;
+              w[4 * blk + 1] = u.y;
+              w[4 * blk + 2] = u.z;
+              w[4 * blk + 3] = u.w;
+            }
+#pragma unroll
+            for (int g = 0; g < static_cast<int>(C::kSfbGroups); ++g) {
+              if constexpr (kBN % 128 != 0)
+                sb[kb * C::kSfbGroups + g] = mid ? w[g + 2] : w[g];
+              else
+                sb[kb * C::kSfbGroups + g] = w[g];
+            }
+          }
+          tmem_st_32x32b_x16(t_quarter + C::kSfaCol + static_cast<uint32_t>(slot) * C::kSfaSlotCols, sa);
+#pragma unroll
+          for (int c = 0; c < static_cast<int>(C::kSfbSlotCols / 8); ++c)
+            tmem_st_32x32b_x8(t_quarter + C::kSfbCol + static_cast<uint32_t>(slot) * C::kSfbSlotCols + c * 8,
+                              sb + 8 * c);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -539,10 +582,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kCG, int kBN, int kAcc, bool kFused>
+template <int kCG, int kBN, int kAcc, bool kFused, bool kMx>
 cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t stream, const DeviceInfo& dev) {
-  using C = Cfg<kCG, kBN, kAcc>;
-  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused>;
+  using C = Cfg<kCG, kBN, kAcc, kMx>;
+  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused, kMx>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -583,11 +626,18 @@ GemmConfig gemm_config(int64_t M, int64_t N) {
   return GemmConfig{1, 192, 2};
 }
 
-cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused,
+cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
                         cudaStream_t stream, const DeviceInfo& dev) {
+  if (mx) {  // MXFP8 operands: the default tile shapes, no fused epilogue
+    if (fused) return cudaErrorInvalidConfiguration;
+    if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2) return launch<2, 192, 2, false, true>(m, p, stream, dev);
+    if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2) return launch<1, 192, 2, false, true>(m, p, stream, dev);
+    return cudaErrorInvalidConfiguration;
+  }
 #define NVFP4_GEMM_CASE(CG, BN, ACC)                                                                          \
   if (c.cta_group == CG && c.tile_n == BN && c.acc_bufs == ACC)                                             \
-    return fused ? launch<CG, BN, ACC, true>(m, p, stream, dev) : launch<CG, BN, ACC, false>(m, p, stream, dev);
+    return fused ? launch<CG, BN, ACC, true, false>(m, p, stream, dev)                                      \
+                 : launch<CG, BN, ACC, false, false>(m, p, stream, dev);
   NVFP4_GEMM_CASE(2, 192, 2)
   NVFP4_GEMM_CASE(1, 192, 2)
   NVFP4_GEMM_CASE(2, 128, 2)

@@ -27,7 +27,7 @@ struct GemmParams {
   int32_t M, N, K;
   int32_t tiles_m, tiles_n, num_tiles;  // tiles_m counts (128 * CTA-group)-row tiles
   int32_t num_kt;  // k-tiles of 256 elements (last one may be partial)
-  int32_t k64;     // K / 64: MMA k-blocks in total, and scale atoms per 128-row block
+  int32_t kblocks; // MMA k-blocks in total: K / 64 (NVFP4) or K / 32 (MXFP8)
   float alpha;
   const float* alpha_scale;   // nullable: if set, the epilogue uses fl(alpha * alpha_scale[0])
   const __nv_bfloat16* bias;  // nullable
@@ -63,6 +63,9 @@ constexpr size_t kDynamicScratchBytes = 8;
 // tmap_x: bf16 [M, K], box 128 rows x 64 columns, 128-byte swizzle.
 cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
                             cudaStream_t stream, const DeviceInfo& dev);
+// MXFP8 (E4M3 codes [M, K], E8M0 scales, one per 32 elements, swizzled).
+cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
+                                  cudaStream_t stream, const DeviceInfo& dev);
 // Same, with g measured on x in the same (cooperative) launch.
 cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, uint8_t* codes,
                                     uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream,
@@ -77,7 +80,8 @@ struct GemmConfig {
   int acc_bufs;   // accumulator buffers in TMEM
 };
 GemmConfig gemm_config(int64_t M, int64_t N);
-cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused,
+// mx: MXFP8 operands (E4M3 codes [rows, K], E8M0 scales) instead of NVFP4.
+cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
                         cudaStream_t stream, const DeviceInfo& dev);
 
 }  // namespace nvfp4

@@ -41,7 +41,7 @@ constexpr uint32_t kQOffBar = kQStages * kQTileBytes;
 constexpr uint32_t kQOffMax = kQOffBar + 2 * kQStages * 8 + 16;  // per-warp maxima of the amax pass
 constexpr uint32_t kQSmemBytes = kQOffMax + 32 * 4 + 1024;        // + alignment slack
 
-template <bool kDynamic>
+template <bool kDynamic, bool kMx>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t M, int64_t K, float g,
                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int64_t tiles_k, int64_t n_tiles,
@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     bool have_scale = !kDynamic;
     float d6 = __fmul_rn(6.0f, g);
     const int64_t katoms = K >> 6;
+    const int64_t mx_katoms = (K / 32 + 3) / 4;  // MXFP8 scale atoms per 128-row block
 
     // Dynamic variant, once per consumer warp (every one of the 16 reaches
     // it exactly once, so the named barriers below always complete): fold
@@ -196,7 +197,47 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
       const int64_t tile = seq_tile(jj);
       const int64_t row = (tile / tiles_k) * kQRows + rloc;
-      const int64_t katom = tile % tiles_k;  // 64-column group = scale atom column
+      const int64_t katom = tile % tiles_k;  // 64-column group of the tile
+      if constexpr (kMx) {
+        // MXFP8: two 32-element blocks -> 64 E4M3 bytes and two E8M0 scale
+        // bytes (scale columns 2*katom, 2*katom + 1: half of a 4-byte word)
+        uint32_t sfh = 0u;
+        uint32_t cw[16];
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          float f[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 u = v[4 * blk + c];
+            f[8 * c + 0] = bf16_lo(u.x);
+            f[8 * c + 1] = bf16_hi(u.x);
+            f[8 * c + 2] = bf16_lo(u.y);
+            f[8 * c + 3] = bf16_hi(u.y);
+            f[8 * c + 4] = bf16_lo(u.z);
+            f[8 * c + 5] = bf16_hi(u.z);
+            f[8 * c + 6] = bf16_lo(u.w);
+            f[8 * c + 7] = bf16_hi(u.w);
+          }
+          uint32_t w[8];
+          sfh |= quantize_mx_block32(f, w) << (8 * blk);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cw[8 * blk + i] = w[i];
+        }
+        if (row < M) {
+          uint8_t* crow = codes + row * K + katom * 64;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(crow + 16 * c) = make_uint4(cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
+        }
+        // rows past M: zero-filled data, amax 0, scale bytes 0 (the padding).
+        // The last tile of a K that is 64 mod 128 also zeroes the two padding
+        // columns of its word.
+        if ((katom & 1) == 0 && katom == tiles_k - 1)
+          *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 2, mx_katoms)) = sfh;
+        else
+          *reinterpret_cast<uint16_t*>(sf + sf_offset(row, katom * 2, mx_katoms)) = static_cast<uint16_t>(sfh);
+        continue;
+      }
       uint32_t sfw = 0u;
       uint32_t cw[8];
 #pragma unroll
@@ -272,10 +313,24 @@ cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, flo
   const int64_t n_tiles = tiles_m * tiles_k;
   const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
   cudaError_t err =
-      cudaFuncSetAttribute(quantize_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+      cudaFuncSetAttribute(quantize_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
   if (err != cudaSuccess) return err;
-  quantize_kernel<false><<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles,
+  quantize_kernel<false, false><<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles,
                                                                    dev.fault, DynamicScaleArgs{});
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
+                                  cudaStream_t stream, const DeviceInfo& dev) {
+  const int64_t tiles_m = (M + kQRows - 1) / kQRows;
+  const int64_t tiles_k = (K + kQCols - 1) / kQCols;
+  const int64_t n_tiles = tiles_m * tiles_k;
+  const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
+  auto kernel = quantize_kernel<false, true>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+  if (err != cudaSuccess) return err;
+  kernel<<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, 0.0f, codes, sf, tiles_k, n_tiles, dev.fault,
+                                                   DynamicScaleArgs{});
   return cudaGetLastError();
 }
 
@@ -286,7 +341,7 @@ cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, in
   const int64_t tiles_k = (K + kQCols - 1) / kQCols;
   const int64_t n_tiles = tiles_m * tiles_k;
   const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
-  auto kernel = quantize_kernel<true>;
+  auto kernel = quantize_kernel<true, false>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
   if (err != cudaSuccess) return err;
   // the grid-wide maximum and the arrival counter start at zero

@@ -22,8 +22,8 @@ def declared_functions():
 def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ("nvfp4_sf_bytes", "nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm",
-              "nvfp4_gemm_quant", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_check_fault",
-              "nvfp4_last_error"):
+              "nvfp4_gemm_quant", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_mxfp8_sf_bytes",
+              "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_check_fault", "nvfp4_last_error"):
         assert n in names
 
 
@@ -99,6 +99,21 @@ def test_dynamic_entry_points_reject_bad_arguments_on_the_host():
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, 1.0, 0, 0, P, 0)   # no g_a
     _expect(F.NVFP4_EALIGN, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, 1.0, P + 1, 0, P, 0)
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, float("nan"), P, 0, P, 0)
+
+
+@pytest.mark.parametrize("rows,k,want", [(4608, 3072, 4608 * 96), (1, 64, 128 * 4), (129, 192, 256 * 8),
+                                         (0, 64, 0), (5, 16, 0), (5, 48, 0)])
+def test_mxfp8_sf_bytes(rows, k, want):
+    assert F.nvfp4_mxfp8_sf_bytes(rows, k) == want
+
+
+def test_mxfp8_entry_points_reject_bad_arguments_on_the_host():
+    _expect(F.NVFP4_EINVAL, F.nvfp4_mxfp8_quantize, 0, 16, 64, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_mxfp8_quantize, P, 16, 96, P, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_mxfp8_quantize, P, 16, 64, P + 4, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_mxfp8_gemm, P, P, P, P, 16, 12, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_mxfp8_gemm, P, P, P, P, 16, 64, 32, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_mxfp8_gemm, P, P, P + 8, P, 16, 64, 64, 1.0, 0, P, 0)
 
 
 def test_calibrate_and_swizzle_reject_bad_arguments_on_the_host():
