@@ -14,3 +14,4 @@ from .nvfp4_ref import (  # noqa: F401  (explicit re-exports for readers)
     sf_offset, sf_padded_shape, swizzle_sf, tensor_amax, unpack_codes, unswizzle_sf,
 )
 from . import mxfp8_ref  # noqa: F401,E402  (the MXFP8 variant: 32-element blocks, E8M0 scales)
+from . import fp8row_ref  # noqa: F401,E402  (row-wise FP8: E4M3 with one fp32 scale per row)
