@@ -489,6 +489,11 @@ def run_ours(args):
     xq8 = F.quantize_mxfp8(x, stream=stream)
     q8_ms = median_ms(lambda: F.quantize_mxfp8(x, out=xq8, stream=stream))
     g8_ms = median_ms(lambda: F.gemm_mxfp8(xq8, wq8, bias=bias, y=y, stream=stream))
+    # row-wise FP8 (W8A8) on the same shape: E4M3 with one fp32 scale per row
+    wr8 = F.quantize_fp8row(w, stream=stream)
+    xr8 = F.quantize_fp8row(x, stream=stream)
+    qr_ms = median_ms(lambda: F.quantize_fp8row(x, out=xr8, stream=stream))
+    gr_ms = median_ms(lambda: F.gemm_fp8row(xr8, wr8, bias=bias, y=y, stream=stream))
     F.nvfp4_check_fault()
     extras = {}
     if world == 1 and not args.no_extras:
@@ -550,6 +555,14 @@ def run_ours(args):
                     "gemm_frac_of_fp8_peak": flops / (g8_ms * 1e-3) / 1e12 / (bf16 * FP8_PER_BF16),
                     "note": "MLP-up shape with MXFP8 operands (E4M3, E8M0 per 32); quantize bytes 2 + 1 + 1/32 "
                             "per element; FP8 peak = measured bf16 burst x 2 (nominal FP8/bf16 dense ratio)"},
+                "fp8row": {
+                    "quantize_ms": qr_ms,
+                    "quantize_gbs": (M * K * 3 + M * 4) / (qr_ms * 1e-3) / 1e9,
+                    "quantize_frac_of_hbm": (M * K * 3 + M * 4) / (qr_ms * 1e-3) / 1e9 / hbm,
+                    "gemm_ms": gr_ms, "gemm_tflops": flops / (gr_ms * 1e-3) / 1e12,
+                    "gemm_frac_of_fp8_peak": flops / (gr_ms * 1e-3) / 1e12 / (bf16 * FP8_PER_BF16),
+                    "note": "MLP-up shape with row-wise FP8 (E4M3, fp32 scale per row of A and of W); quantize "
+                            "bytes 2 + 1 per element + 4 per row"},
                 **extras,
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

@@ -304,6 +304,42 @@ nvfp4_status nvfp4_mxfp8_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_
                               float alpha, const void* bias, void* y, void* stream);
 
 /*
+ * ------------------------------------------------------------------------
+ * Row-wise FP8 (W8A8) variant (BFL doc, `fp8r` bullet and "Kernels" row
+ * `fp8r`: an E4M3 `weight` with one fp32 `weight_scale` per row;
+ * activations quantized to E4M3 row by row at run time; the GEMM applies the
+ * row scales).  No block scales, no per-tensor scale.
+ * ------------------------------------------------------------------------
+ */
+
+/*
+ * bf16 -> row-wise FP8, for activations at run time (and for weights once):
+ *     s[m] = fl(amax(|x[m, :]|) / 448)
+ *     code = E4M3_satfinite(fl(x[m, k] / s[m]))   (RNE, +-448)
+ *   a row of zeros gets s = 0 and the codes of +-0.
+ *   x      [M, K] bf16, finite
+ *   codes  [M, K] uint8 E4M3, written;  scale  [M] fp32, written
+ * M >= 1, K % 64 == 0, all pointers 16-byte aligned.
+ * Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_fp8row_quantize(const void* x, int64_t M, int64_t K,
+                                   uint8_t* codes, float* scale, void* stream);
+
+/*
+ * Row-wise FP8 GEMM on the tensor cores (tcgen05, kind::f8f6f4, E4M3 x E4M3
+ * -> fp32 accumulation), scales folded into the epilogue:
+ *     y[m, n] = bf16_rn( fl(a_scale[m] * b_scale[n]) * acc[m, n] + bias[n] )
+ *   a [M, K] codes, a_scale [M];  b [N, K] codes (the weight, PyTorch
+ *   [out, in]), b_scale [N] (16-byte aligned);  bias [N] bf16 or NULL;
+ *   y [M, N] bf16, written.
+ * M >= 1, N >= 8 with N % 8 == 0, K % 64 == 0.  Errors: EINVAL, EALIGN,
+ * EARCH, ECUDA; a barrier time-out records NVFP4_ETIMEOUT.
+ */
+nvfp4_status nvfp4_fp8row_gemm(const uint8_t* a, const float* a_scale, const uint8_t* b,
+                               const float* b_scale, int64_t M, int64_t N, int64_t K,
+                               const void* bias, void* y, void* stream);
+
+/*
  * Synchronize the current device, then read and clear its fault word.
  * Returns NVFP4_ETIMEOUT if any kernel of this library gave up on a barrier
  * wait since the last check, NVFP4_ECUDA if the synchronize failed, else

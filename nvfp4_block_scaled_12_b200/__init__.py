@@ -64,10 +64,13 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_mxfp8_sf_bytes.restype = ctypes.c_size_t
     lib.nvfp4_mxfp8_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
     lib.nvfp4_mxfp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
+    lib.nvfp4_fp8row_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+    lib.nvfp4_fp8row_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
-                 "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_check_fault"):
+                 "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
+                 "nvfp4_check_fault"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -148,6 +151,15 @@ def nvfp4_mxfp8_quantize(x: int, M: int, K: int, codes: int, sf: int, stream: in
 def nvfp4_mxfp8_gemm(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha: float, bias: int, y: int,
                      stream: int) -> None:
     _check(library().nvfp4_mxfp8_gemm(a, sfa, b, sfb, M, N, K, alpha, bias or None, y, stream))
+
+
+def nvfp4_fp8row_quantize(x: int, M: int, K: int, codes: int, scale: int, stream: int) -> None:
+    _check(library().nvfp4_fp8row_quantize(x, M, K, codes, scale, stream))
+
+
+def nvfp4_fp8row_gemm(a: int, a_scale: int, b: int, b_scale: int, M: int, N: int, K: int, bias: int, y: int,
+                      stream: int) -> None:
+    _check(library().nvfp4_fp8row_gemm(a, a_scale, b, b_scale, M, N, K, bias or None, y, stream))
 
 
 def nvfp4_check_fault() -> None:
@@ -285,6 +297,43 @@ def gemm_mxfp8(a: MXFP8Tensor, b: MXFP8Tensor, bias=None, alpha: float = 1.0, y=
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
     nvfp4_mxfp8_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias),
                      _ptr(y), _stream(stream))
+    return y
+
+
+@dataclass
+class FP8RowTensor:
+    """A [rows, k] row-wise FP8 tensor on the GPU: E4M3 codes and one fp32
+    scale per row."""
+    codes: "object"   # uint8 [rows, k]
+    scale: "object"   # float32 [rows]
+    rows: int
+    k: int
+
+
+def quantize_fp8row(x, out: Optional[FP8RowTensor] = None, stream=None) -> FP8RowTensor:
+    """Quantize bf16 ``x`` [M, K] to E4M3 with one absmax scale per row."""
+    torch = _torch()
+    M, K = x.shape
+    _need(x, torch.bfloat16, None, "x")
+    if out is None:
+        out = FP8RowTensor(torch.empty(M, K, dtype=torch.uint8, device=x.device),
+                           torch.empty(M, dtype=torch.float32, device=x.device), M, K)
+    nvfp4_fp8row_quantize(_ptr(x), M, K, _ptr(out.codes), _ptr(out.scale), _stream(stream))
+    return out
+
+
+def gemm_fp8row(a: FP8RowTensor, b: FP8RowTensor, bias=None, y=None, stream=None):
+    """y = bf16(a_scale[m] * b_scale[n] * a_q @ b_q^T + bias)."""
+    torch = _torch()
+    if a.k != b.k:
+        raise ValueError("K mismatch")
+    M, N, K = a.rows, b.rows, a.k
+    if bias is not None:
+        _need(bias, torch.bfloat16, (N,), "bias")
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    nvfp4_fp8row_gemm(_ptr(a.codes), _ptr(a.scale), _ptr(b.codes), _ptr(b.scale), M, N, K, _ptr(bias), _ptr(y),
+                      _stream(stream))
     return y
 
 

@@ -172,10 +172,11 @@ bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
 
 // Checks shared by the two GEMM entry points; fills the operand part of p
 // and the operand tensor maps.
-// mx: MXFP8 operands (one E4M3 byte per element, E8M0 scales per 32).
+// mx: 8-bit operands (one E4M3 byte per element), with E8M0 scales per 32
+// (MXFP8) or, with row, one fp32 scale per row passed as sfa / sfb.
 nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
                          int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, GemmTensorMaps* maps,
-                         GemmConfig* cfg, const DeviceInfo** dev, bool mx = false) {
+                         GemmConfig* cfg, const DeviceInfo** dev, bool mx = false, bool row = false) {
   if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
   if (M < 1 || M > INT32_MAX / 2) return fail(NVFP4_EINVAL, "M=%lld out of range", (long long)M);
   if (N < 8 || N % 8 != 0 || N > INT32_MAX / 2)
@@ -212,9 +213,9 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   p->pf_ptr[1] = a;
   p->pf_bytes[1] = static_cast<uint64_t>(M) * static_cast<uint64_t>(row_bytes);
   p->pf_ptr[2] = sfb;
-  p->pf_bytes[2] = mx ? nvfp4_mxfp8_sf_bytes(N, K) : nvfp4_sf_bytes(N, K);
+  p->pf_bytes[2] = row ? static_cast<uint64_t>(N) * 4 : mx ? nvfp4_mxfp8_sf_bytes(N, K) : nvfp4_sf_bytes(N, K);
   p->pf_ptr[3] = sfa;
-  p->pf_bytes[3] = mx ? nvfp4_mxfp8_sf_bytes(M, K) : nvfp4_sf_bytes(M, K);
+  p->pf_bytes[3] = row ? static_cast<uint64_t>(M) * 4 : mx ? nvfp4_mxfp8_sf_bytes(M, K) : nvfp4_sf_bytes(M, K);
 
   st = make_tmap(&maps->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, row_bytes, M, row_bytes, 128, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B, "A");
@@ -222,6 +223,11 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   st = make_tmap(&maps->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, row_bytes, N, row_bytes, 128, bn / cg,
                  CU_TENSOR_MAP_SWIZZLE_128B, "B");
   if (st != NVFP4_OK) return st;
+  if (row) {  // no block scales: the kernel reads the row scales in its epilogue
+    p->row_scale = reinterpret_cast<const float*>(sfa);
+    p->col_scale = reinterpret_cast<const float*>(sfb);
+    return NVFP4_OK;
+  }
   // scale atoms per 128-row block, and atoms per k-tile
   const int64_t atoms = mx ? (K / 32 + 3) / 4 : K / 64;
   const uint32_t box_atoms = mx ? 1u : 4u;
@@ -281,6 +287,40 @@ nvfp4_status nvfp4_mxfp8_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_
   if (st != NVFP4_OK) return st;
   cudaError_t e = launch_gemm(maps, p, cg, false, true, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "mxfp8 gemm launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_fp8row_quantize(const void* x, int64_t M, int64_t K, uint8_t* codes, float* scale,
+                                   void* stream) {
+  if (!x || !codes || !scale) return fail(NVFP4_EINVAL, "null pointer");
+  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
+  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scale))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_quantize_rowwise(x, M, K, codes, scale, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "row-wise fp8 quantize launch");
+  return ok();
+}
+
+nvfp4_status nvfp4_fp8row_gemm(const uint8_t* a, const float* a_scale, const uint8_t* b, const float* b_scale,
+                               int64_t M, int64_t N, int64_t K, const void* bias, void* y, void* stream) {
+  if (!y) return fail(NVFP4_EINVAL, "null output pointer");
+  if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
+  GemmParams p;
+  GemmTensorMaps maps;
+  GemmConfig cg;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, reinterpret_cast<const uint8_t*>(a_scale), b,
+                                reinterpret_cast<const uint8_t*>(b_scale), M, N, K, 1.0f, bias, &p, &maps, &cg, &dev,
+                                true, true);
+  if (st != NVFP4_OK) return st;
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm(maps, p, cg, false, true, static_cast<cudaStream_t>(stream), *dev, true);
+  if (e != cudaSuccess) return cuda_fail(e, "row-wise fp8 gemm launch");
   return ok();
 }
 

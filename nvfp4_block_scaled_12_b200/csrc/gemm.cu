@@ -53,20 +53,22 @@ constexpr int kProducers = 2;  // warps 0 and 10
 constexpr uint32_t kTmemCols = 512;
 
 // kCG: CTAs per tile; kBN: tile width; kAcc: accumulator buffers in TMEM;
-// kMx: MXFP8 operands (E4M3, one E8M0 scale per 32 elements) instead of NVFP4.
-template <int kCG, int kBN, int kAcc, bool kMx>
+// kMx: 8-bit E4M3 operands (K = 32 per MMA) instead of NVFP4; with kRow they
+// carry no block scales at all (row-wise FP8: one scale per row of A and of
+// B, applied in the epilogue), otherwise one E8M0 scale per 32 elements.
+template <int kCG, int kBN, int kAcc, bool kMx, bool kRow = false>
 struct Cfg {
   // 512-byte scale atoms (128 rows x 4 scale columns) per 128-row block and
   // k-tile: NVFP4's k-tile is 4 MMA k-blocks of 64 elements with one 4-scale
   // word per row each; MXFP8's is 4 k-blocks of 32 whose scales share one word.
   static constexpr int kAtoms = kMx ? 1 : 4;
-  static constexpr uint32_t kSfaBytes = kAtoms * 512;
+  static constexpr uint32_t kSfaBytes = kRow ? 0 : kAtoms * 512;
   static constexpr int kBNc = kBN / kCG;  // B rows per CTA
   static constexpr uint32_t kBBytes = kBNc * kBKBytes;
   static constexpr int kChunks = kBN / 32;
   // 128-row scale blocks a B tile can touch (a 192-wide tile may start mid-block)
   static constexpr int kSfbBlocks = kBN % 128 == 0 ? kBN / 128 : kBN / 128 + 1;
-  static constexpr uint32_t kSfbBytes = kSfbBlocks * kAtoms * 512;
+  static constexpr uint32_t kSfbBytes = kRow ? 0 : kSfbBlocks * kAtoms * 512;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStagesFit = (224 * 1024 - 4 * 2 * 2048) / kStageBytes;
   // a multiple of the producer count: each stage then has a single producer
@@ -132,13 +134,14 @@ __device__ __forceinline__ void store_chunk_bf16(const CUtensorMap* tmap, uint8_
   }
 }
 
-template <int kCG, int kBN, int kAcc, bool kFused, bool kMx>
+template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ GemmParams p) {
-  using C = Cfg<kCG, kBN, kAcc, kMx>;
+  using C = Cfg<kCG, kBN, kAcc, kMx, kRow>;
   static_assert(!(kFused && kMx), "the fused quantize epilogue writes NVFP4 after an NVFP4 GEMM");
+  static_assert(!kRow || kMx, "row-wise FP8 uses the 8-bit operand layout");
   constexpr int S = C::kStages;
   constexpr int R = C::kSfSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -162,7 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1 + 4 * kCG);  // the producer's expect_tx and every scale mover of the group
+      // the producer's expect_tx and every scale mover of the group
+      mbar_init(&full[s], kRow ? 1 : 1 + 4 * kCG);
       mbar_init(&empty[s], 1);
       mbar_init(&sfin[s], 1);
     }
@@ -177,8 +181,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
-    prefetch_tmap(&tmap_sfa);
-    prefetch_tmap(&tmap_sfb);
+    if (!kRow) {
+      prefetch_tmap(&tmap_sfa);
+      prefetch_tmap(&tmap_sfb);
+    }
     prefetch_tmap(&tmap_y);
   }
   if (warp == 1) {
@@ -243,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n0 = (tile / p.tiles_m) * kBN;
         const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
         if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
-        mbar_arrive_expect_tx(&sfin[stage], C::kSfaBytes + C::kSfbBytes);
+        if (!kRow) mbar_arrive_expect_tx(&sfin[stage], C::kSfaBytes + C::kSfbBytes);
         uint8_t* sa = smem + C::kOffA + stage * kABytes;
         uint8_t* sb = smem + C::kOffB + stage * C::kBBytes;
         if (kCG == 2) {
@@ -254,8 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sa, &tmap_a, &full[stage], kt * kBKBytes, row_block * 128);
           tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
         }
-        tma_load_3d(smem + C::kOffSfa + stage * C::kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * C::kAtoms, row_block);
-        tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * C::kAtoms, n0 >> 7);
+        if (!kRow) {
+          tma_load_3d(smem + C::kOffSfa + stage * C::kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * C::kAtoms, row_block);
+          tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * C::kAtoms, n0 >> 7);
+        }
       }
       if (fault != 0u) {
         *abort_flag = 1;
@@ -263,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int64_t i = j - kProducers; i >= 0 && i >= j - S; i -= kProducers) {
           const int stage = static_cast<int>(i % S);
           const uint32_t phase = static_cast<uint32_t>((i / S) & 1);
-          mbar_wait(&sfin[stage], phase, nullptr);
+          if (!kRow) mbar_wait(&sfin[stage], phase, nullptr);
           if (leader) mbar_wait(&full[stage], phase, nullptr);
         }
       }
@@ -275,7 +283,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // byte kb of the k-tile's scale words (named in the descriptor and in
       // the top two bits of the scale addresses)
       auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb, int kb, uint32_t accum) {
-        if constexpr (kMx) {
+        if constexpr (kRow) {
+          constexpr uint32_t idesc = idesc_f8(128 * kCG, kBN);
+          if (kCG == 2)
+            tc_mma_f8_pair(d, ad, bd, idesc, accum);
+          else
+            tc_mma_f8(d, ad, bd, idesc, accum);
+        } else if constexpr (kMx) {
           const uint32_t idesc = idesc_mxf8(128 * kCG, kBN, static_cast<uint32_t>(kb));
           const uint32_t sel = static_cast<uint32_t>(kb) << 30;
           if (kCG == 2)
@@ -352,6 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(drain, 0u, nullptr)) fault |= kFaultDrainWait;
     }
     __syncwarp();
+  } else if (warp >= 6 && kRow) {
+    // row-wise FP8 has no block scales to move
   } else if (warp >= 6) {
     // ------------------------------------------------------------ scale movers (warps 6-9)
     const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter of this warp
@@ -522,8 +538,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           bias[8 * g + 7] = bf16_hi(b.w);
         }
         float v[32];
+        if constexpr (kRow) {
+          // row-wise FP8: y = fl(s_a[row] * s_b[n]) * acc + bias
+          const float sa = row < p.M ? __ldg(p.row_scale + row) : 0.0f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = round_bf16(fmaf(alpha, __uint_as_float(r[j]), bias[j]));
+          for (int g = 0; g < 8; ++g) {
+            float4 cs = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (n + 4 * g < p.N) cs = __ldg(reinterpret_cast<const float4*>(p.col_scale + n + 4 * g));
+            v[4 * g + 0] = round_bf16(fmaf(__fmul_rn(sa, cs.x), __uint_as_float(r[4 * g + 0]), bias[4 * g + 0]));
+            v[4 * g + 1] = round_bf16(fmaf(__fmul_rn(sa, cs.y), __uint_as_float(r[4 * g + 1]), bias[4 * g + 1]));
+            v[4 * g + 2] = round_bf16(fmaf(__fmul_rn(sa, cs.z), __uint_as_float(r[4 * g + 2]), bias[4 * g + 2]));
+            v[4 * g + 3] = round_bf16(fmaf(__fmul_rn(sa, cs.w), __uint_as_float(r[4 * g + 3]), bias[4 * g + 3]));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = round_bf16(fmaf(alpha, __uint_as_float(r[j]), bias[j]));
+        }
         if (kFused && act == NVFP4_ACT_GELU_TANH) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = round_bf16(gelu_tanh_f32(v[j]));
@@ -582,10 +612,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kCG, int kBN, int kAcc, bool kFused, bool kMx>
+template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow = false>
 cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t stream, const DeviceInfo& dev) {
-  using C = Cfg<kCG, kBN, kAcc, kMx>;
-  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused, kMx>;
+  using C = Cfg<kCG, kBN, kAcc, kMx, kRow>;
+  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused, kMx, kRow>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -627,7 +657,15 @@ GemmConfig gemm_config(int64_t M, int64_t N) {
 }
 
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
-                        cudaStream_t stream, const DeviceInfo& dev) {
+                        cudaStream_t stream, const DeviceInfo& dev, bool row) {
+  if (row) {  // row-wise FP8: the default tile shapes, no fused epilogue
+    if (fused || !mx) return cudaErrorInvalidConfiguration;
+    if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2)
+      return launch<2, 192, 2, false, true, true>(m, p, stream, dev);
+    if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2)
+      return launch<1, 192, 2, false, true, true>(m, p, stream, dev);
+    return cudaErrorInvalidConfiguration;
+  }
   if (mx) {  // MXFP8 operands: the default tile shapes, no fused epilogue
     if (fused) return cudaErrorInvalidConfiguration;
     if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2) return launch<2, 192, 2, false, true>(m, p, stream, dev);

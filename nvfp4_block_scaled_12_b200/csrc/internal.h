@@ -30,6 +30,8 @@ struct GemmParams {
   int32_t kblocks; // MMA k-blocks in total: K / 64 (NVFP4) or K / 32 (MXFP8)
   float alpha;
   const float* alpha_scale;   // nullable: if set, the epilogue uses fl(alpha * alpha_scale[0])
+  const float* row_scale;     // row-wise FP8: [M] scales of A's rows
+  const float* col_scale;     // row-wise FP8: [N] scales of B's rows (output columns)
   const __nv_bfloat16* bias;  // nullable
   unsigned* fault;
   // operand byte ranges prefetched into L2 at kernel start (A, B, SFA, SFB)
@@ -81,7 +83,11 @@ struct GemmConfig {
 };
 GemmConfig gemm_config(int64_t M, int64_t N);
 // mx: MXFP8 operands (E4M3 codes [rows, K], E8M0 scales) instead of NVFP4.
+// row: row-wise FP8 (8-bit operands without block scales; requires mx).
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
-                        cudaStream_t stream, const DeviceInfo& dev);
+                        cudaStream_t stream, const DeviceInfo& dev, bool row = false);
+// Row-wise FP8 quantize: x bf16 [M, K] -> codes [M, K] E4M3, scale [M] fp32.
+cudaError_t launch_quantize_rowwise(const void* x, int64_t M, int64_t K, uint8_t* codes, float* scale,
+                                    cudaStream_t stream);
 
 }  // namespace nvfp4
