@@ -54,6 +54,10 @@ Pins (the tests that tie each function to something other than itself):
                                  triple-loop brute force)
   gelu_tanh                      tests/test_oracle_gemm.py (torch gelu 'tanh'
                                  in fp64, odd-part identity)
+  dequantize_to_bf16 / linear_w4a16_ref
+                                 tests/test_oracle_gemm.py (power-of-two
+                                 scales against ml_dtypes decoding, the
+                                 rounding bound, torch's bf16 conversion)
 """
 from __future__ import annotations
 
@@ -317,6 +321,32 @@ def unswizzle_sf(sf_swz, rows: int, k: int) -> np.ndarray:
 # ----------------------------------------------------------------------------
 # GEMM with dequant epilogue
 # ----------------------------------------------------------------------------
+
+def dequantize_to_bf16(codes, sf, g) -> np.ndarray:
+    """Weights dequantized to the bf16 compute dtype, as the W4A16 path does on
+    every forward ("BFL (fp8r / nvfp4)" doc, section "Kernels", last
+    paragraph): ``v = fl32(fl32(e2m1(q) * e4m3(s)) * g)`` -- the first product
+    is exact in fp32 -- then rounded to bf16 (RNE).  Returns float32 values
+    that are exactly bf16, shape [rows, K]."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    rows = codes.shape[0]
+    q = e2m1_decode(unpack_codes(codes)).astype(np.float32)            # exact
+    s = e4m3_decode(np.asarray(sf, np.uint8)).astype(np.float32)       # exact
+    prod = (q.reshape(rows, -1, BLOCK) * s[:, :, None]).astype(np.float32)   # exact (<= 3 x 4 significant bits)
+    v = (prod * np.float32(g)).astype(np.float32).reshape(rows, -1)    # one fp32 rounding
+    return round_to_bf16(v.astype(np.float64)).astype(np.float32)
+
+
+def linear_w4a16_ref(x_bf16, w_codes, w_sf, g_w, bias=None) -> np.ndarray:
+    """``y = x @ w_bf16^T + bias`` in float64 with ``w_bf16 =
+    dequantize_to_bf16(w)``: the regular linear the W4A16 path runs (the
+    activations stay bf16)."""
+    w = dequantize_to_bf16(w_codes, w_sf, g_w).astype(np.float64)
+    y = np.asarray(x_bf16, dtype=np.float64) @ w.T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y
+
 
 def gemm_ref(a_codes, a_sf, g_a, b_codes, b_sf, g_b, bias=None) -> np.ndarray:
     """``y[m, n] = (g_a * g_b) * sum_k a_hat[m, k] * b_hat[n, k] + bias[n]`` in

@@ -119,3 +119,47 @@ def test_global_scale_is_amax_over_2688(amax):
     assert g.dtype == np.float32
     assert g == np.float32(np.float32(amax) / np.float32(2688.0))
     assert abs(float(g) * 2688.0 / amax - 1) < 1e-6
+
+
+# --------------------------------------------------------------------------
+# W4A16: weights dequantized to bf16, regular linear
+# --------------------------------------------------------------------------
+
+def test_dequantize_to_bf16_with_power_of_two_scale_is_the_exact_product_rounded():
+    # with g a power of two every fp32 step is exact, so the result is the
+    # bf16 rounding (torch's) of e2m1(code) * e4m3(scale) * g decoded by ml_dtypes
+    rng = np.random.default_rng(60)
+    rows, K = 40, 256
+    codes = rng.integers(0, 256, (rows, K // 2)).astype(np.uint8)
+    sf = rng.integers(0, 127, (rows, K // 16)).astype(np.uint8)
+    for g in (1.0, 2.0 ** -7, 2.0 ** 12):
+        q = O.unpack_codes(codes)
+        exact = (q.view(F4).astype(np.float64) * np.repeat(sf.view(F8).astype(np.float64), 16, axis=1) * g)
+        want = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16).float().numpy()
+        assert np.array_equal(O.dequantize_to_bf16(codes, sf, g), want)
+
+
+def test_dequantize_to_bf16_rounding_bound():
+    rng = np.random.default_rng(61)
+    codes = rng.integers(0, 256, (64, 64)).astype(np.uint8)
+    sf = rng.integers(1, 127, (64, 8)).astype(np.uint8)
+    g = 0.00731
+    v = O.dequantize_to_bf16(codes, sf, g)
+    exact = O.dequantize(codes, sf, g)   # fp64
+    # fp32 then bf16 rounding: within half a bf16 ulp plus half an fp32 ulp
+    bound = np.abs(exact) * (2.0 ** -8 + 2.0 ** -24) + 1e-45
+    assert np.all(np.abs(v - exact) <= bound)
+
+
+def test_linear_w4a16_is_the_bf16_linear_of_the_dequantized_weight():
+    rng = np.random.default_rng(62)
+    x = O.round_to_bf16(rng.standard_normal((5, 64))).astype(np.float32)
+    codes = rng.integers(0, 256, (7, 32)).astype(np.uint8)
+    sf = rng.integers(40, 60, (7, 4)).astype(np.uint8)
+    bias = rng.standard_normal(7)
+    y = O.linear_w4a16_ref(x, codes, sf, 0.5, bias)
+    w = O.dequantize_to_bf16(codes, sf, 0.5)
+    for m in range(5):
+        for n in range(7):
+            assert y[m, n] == pytest.approx(sum(float(x[m, k]) * float(w[n, k]) for k in range(64)) + bias[n],
+                                            rel=1e-12, abs=1e-12)
