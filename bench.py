@@ -336,13 +336,15 @@ def extra_workloads(F, torch, synth, device, stream, median_ms, hbm, fp4_peak):
         y = torch.empty(wl.m, wl.n, dtype=torch.bfloat16, device=device)
         tq = median_ms(lambda: F.quantize(x, g, out=xq, stream=stream))
         tg = median_ms(lambda: F.gemm(xq, wq, y=y, stream=stream))
+        w16 = F.dequantize(wq, stream=stream)
+        tw = median_ms(lambda: F.linear_w4a16(x, wq, None, w_bf16=w16, stream=stream))
         flops = 2 * wl.m * wl.n * wl.k
         # min(compute, memory) roofline: A + B + scales in, Y out
         bytes_ = wl.m * wl.k / 2 + wl.n * wl.k / 2 + (wl.m + wl.n) * wl.k / 16 + wl.m * wl.n * 2
         t_roof = max(flops / (fp4_peak * 1e12), bytes_ / (hbm * 1e9)) * 1e3
         sweep.append({"m": wl.m, "quantize_ms": tq, "gemm_ms": tg, "gemm_tflops": flops / (tg * 1e-3) / 1e12,
-                      "frac_of_roofline": t_roof / tg})
-        del x, xq, w, wq, y
+                      "frac_of_roofline": t_roof / tg, "w4a16_linear_ms": tw})
+        del x, xq, w, wq, y, w16
     out["proj_sweep_k3072_n3072"] = sweep
     return out
 
@@ -494,6 +496,11 @@ def run_ours(args):
     xr8 = F.quantize_fp8row(x, stream=stream)
     qr_ms = median_ms(lambda: F.quantize_fp8row(x, out=xr8, stream=stream))
     gr_ms = median_ms(lambda: F.gemm_fp8row(xr8, wr8, bias=bias, y=y, stream=stream))
+    # W4A16: the weight dequantized to bf16 by this library, then a regular
+    # bf16 linear (a library GEMM) on the unquantized activations
+    w16 = F.dequantize(wq, stream=stream)
+    dq_ms = median_ms(lambda: F.dequantize(wq, out=w16, stream=stream))
+    lw_ms = median_ms(lambda: F.linear_w4a16(x, wq, bias, w_bf16=w16, stream=stream))
     F.nvfp4_check_fault()
     extras = {}
     if world == 1 and not args.no_extras:
@@ -563,6 +570,13 @@ def run_ours(args):
                     "gemm_frac_of_fp8_peak": flops / (gr_ms * 1e-3) / 1e12 / (bf16 * FP8_PER_BF16),
                     "note": "MLP-up shape with row-wise FP8 (E4M3, fp32 scale per row of A and of W); quantize "
                             "bytes 2 + 1 per element + 4 per row"},
+                "w4a16": {
+                    "dequantize_ms": dq_ms,
+                    "dequantize_gbs": N * K * QUANT_BYTES_PER_ELEM / (dq_ms * 1e-3) / 1e9,
+                    "dequantize_frac_of_hbm": N * K * QUANT_BYTES_PER_ELEM / (dq_ms * 1e-3) / 1e9 / hbm,
+                    "linear_ms": lw_ms, "linear_tflops": flops / (lw_ms * 1e-3) / 1e12,
+                    "note": "MLP-up weight [12288,3072] NVFP4 -> bf16 (0.5 + 1/16 in, 2 out per element), then "
+                            "torch linear (cuBLAS bf16) on bf16 activations; linear_ms includes the dequantize"},
                 **extras,
             },
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

@@ -340,6 +340,21 @@ nvfp4_status nvfp4_fp8row_gemm(const uint8_t* a, const float* a_scale, const uin
                                const void* bias, void* y, void* stream);
 
 /*
+ * W4A16 path (BFL doc, "Kernels", last paragraph: where the fused kernels do
+ * not run, the NVFP4 weights are dequantized to the compute dtype on every
+ * forward and the layer runs as a regular linear with bf16 activations):
+ * NVFP4 -> bf16,
+ *     out[r, k] = bf16_rn( fl( fl(e2m1(code) * e4m3(scale)) * g ) )
+ * (the first product is exact in fp32).  The linear itself is a plain bf16
+ * GEMM (a library GEMM), not part of this library.
+ *   codes [rows, K/2], sf swizzled nvfp4_sf_bytes(rows, K), g finite;
+ *   out   [rows, K] bf16, written.
+ * rows >= 1, K % 64 == 0.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, float g,
+                              int64_t rows, int64_t K, void* out, void* stream);
+
+/*
  * Synchronize the current device, then read and clear its fault word.
  * Returns NVFP4_ETIMEOUT if any kernel of this library gave up on a barrier
  * wait since the last check, NVFP4_ECUDA if the synchronize failed, else

@@ -66,11 +66,12 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_mxfp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
     lib.nvfp4_fp8row_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
     lib.nvfp4_fp8row_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
+    lib.nvfp4_dequantize.argtypes = [vp, vp, f32, i64, i64, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
                  "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
-                 "nvfp4_check_fault"):
+                 "nvfp4_dequantize", "nvfp4_check_fault"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -160,6 +161,10 @@ def nvfp4_fp8row_quantize(x: int, M: int, K: int, codes: int, scale: int, stream
 def nvfp4_fp8row_gemm(a: int, a_scale: int, b: int, b_scale: int, M: int, N: int, K: int, bias: int, y: int,
                       stream: int) -> None:
     _check(library().nvfp4_fp8row_gemm(a, a_scale, b, b_scale, M, N, K, bias or None, y, stream))
+
+
+def nvfp4_dequantize(codes: int, sf: int, g: float, rows: int, K: int, out: int, stream: int) -> None:
+    _check(library().nvfp4_dequantize(codes, sf, g, rows, K, out, stream))
 
 
 def nvfp4_check_fault() -> None:
@@ -335,6 +340,24 @@ def gemm_fp8row(a: FP8RowTensor, b: FP8RowTensor, bias=None, y=None, stream=None
     nvfp4_fp8row_gemm(_ptr(a.codes), _ptr(a.scale), _ptr(b.codes), _ptr(b.scale), M, N, K, _ptr(bias), _ptr(y),
                       _stream(stream))
     return y
+
+
+def dequantize(t: NVFP4Tensor, out=None, stream=None):
+    """NVFP4 tensor -> bf16 [rows, k] (the W4A16 path's weight)."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(t.rows, t.k, dtype=torch.bfloat16, device=t.codes.device)
+    nvfp4_dequantize(_ptr(t.codes), _ptr(t.sf), float(t.g), t.rows, t.k, _ptr(out), _stream(stream))
+    return out
+
+
+def linear_w4a16(x, w: NVFP4Tensor, bias=None, w_bf16=None, stream=None):
+    """W4A16 linear: the NVFP4 weight dequantized to bf16 by this library,
+    then a regular bf16 linear (a library GEMM) on the unquantized
+    activations."""
+    torch = _torch()
+    w_bf16 = dequantize(w, out=w_bf16, stream=stream)
+    return torch.nn.functional.linear(x, w_bf16, bias)
 
 
 def swizzle_sf(sf_linear, rows: int, k: int, stream=None):

@@ -324,6 +324,22 @@ nvfp4_status nvfp4_fp8row_gemm(const uint8_t* a, const float* a_scale, const uin
   return ok();
 }
 
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, float g, int64_t rows, int64_t K, void* out,
+                              void* stream) {
+  if (!codes || !sf || !out) return fail(NVFP4_EINVAL, "null pointer");
+  if (rows < 1) return fail(NVFP4_EINVAL, "rows=%lld must be >= 1", (long long)rows);
+  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (!finite_f(g)) return fail(NVFP4_EINVAL, "g must be finite");
+  if (!aligned16(codes) || !aligned16(sf) || !aligned16(out))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_dequantize(codes, sf, g, rows, K, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return ok();
+}
+
 size_t nvfp4_sf_bytes(int64_t rows, int64_t k) {
   if (rows < 1 || k < 16 || k % 16 != 0) return 0;
   const int64_t rp = (rows + 127) / 128 * 128;

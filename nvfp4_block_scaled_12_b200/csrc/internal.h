@@ -86,6 +86,9 @@ GemmConfig gemm_config(int64_t M, int64_t N);
 // row: row-wise FP8 (8-bit operands without block scales; requires mx).
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
                         cudaStream_t stream, const DeviceInfo& dev, bool row = false);
+// NVFP4 [rows, K] (codes, swizzled scales, g) -> bf16 [rows, K].
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* sf, float g, int64_t rows, int64_t K, void* out,
+                              cudaStream_t stream);
 // Row-wise FP8 quantize: x bf16 [M, K] -> codes [M, K] E4M3, scale [M] fp32.
 cudaError_t launch_quantize_rowwise(const void* x, int64_t M, int64_t K, uint8_t* codes, float* scale,
                                     cudaStream_t stream);

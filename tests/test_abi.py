@@ -24,7 +24,7 @@ def test_header_declares_the_expected_entry_points():
     for n in ("nvfp4_sf_bytes", "nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm",
               "nvfp4_gemm_quant", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_mxfp8_sf_bytes",
               "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
-              "nvfp4_check_fault", "nvfp4_last_error"):
+              "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_last_error"):
         assert n in names
 
 
@@ -123,6 +123,13 @@ def test_fp8row_entry_points_reject_bad_arguments_on_the_host():
     _expect(F.NVFP4_EALIGN, F.nvfp4_fp8row_quantize, P, 4, 64, P, P + 4, 0)
     _expect(F.NVFP4_EINVAL, F.nvfp4_fp8row_gemm, P, P, P, P, 16, 12, 64, 0, P, 0)
     _expect(F.NVFP4_EALIGN, F.nvfp4_fp8row_gemm, P, P, P, P + 4, 16, 64, 64, 0, P, 0)
+
+
+def test_dequantize_rejects_bad_arguments_on_the_host():
+    _expect(F.NVFP4_EINVAL, F.nvfp4_dequantize, P, P, 1.0, 0, 64, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_dequantize, P, P, 1.0, 4, 48, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_dequantize, P, P, float("inf"), 4, 64, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_dequantize, P, P, 1.0, 4, 64, P + 2, 0)
 
 
 def test_calibrate_and_swizzle_reject_bad_arguments_on_the_host():
