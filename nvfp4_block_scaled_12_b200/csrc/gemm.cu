@@ -382,20 +382,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       // a 192-wide tile that starts at row 64 of a 128-row scale block
       const bool mid = ((tile / p.tiles_m) * kBN & 127) != 0;
       for (int kt = 0; kt < p.num_kt; ++kt, ++j) {
-        bool got = mbar_wait(&sfin[stage], phase, abort_flag);
-        if (got && j >= R) {
-          got = mbar_wait(&empty[lag_stage], lag_phase, abort_flag);
-          if (++lag_stage == S) {
-            lag_stage = 0;
-            lag_phase ^= 1u;
-          }
-        }
+        const bool landed = mbar_wait(&sfin[stage], phase, abort_flag);
         __syncwarp();
-        if (!__all_sync(0xffffffffu, got)) {
+        if (!__all_sync(0xffffffffu, landed)) {
           fault = kFaultMmaWait;
           break;
         }
-        tc_fence_after();
+        // The scales are read into registers first; only the TMEM stores wait
+        // for slot j % R to be free (the commit of k-tile j - R).
+        auto slot_free = [&]() {
+          bool ok = true;
+          if (j >= R) {
+            ok = mbar_wait(&empty[lag_stage], lag_phase, abort_flag);
+            if (++lag_stage == S) {
+              lag_stage = 0;
+              lag_phase ^= 1u;
+            }
+          }
+          __syncwarp();
+          ok = __all_sync(0xffffffffu, ok);
+          tc_fence_after();
+          return ok;
+        };
         // All loads first (atoms past K arrived zero-filled), then a few wide
         // stores: a shared load is not reordered across a tcgen05.st.
         const uint8_t* ssfa = smem + C::kOffSfa + stage * C::kSfaBytes + lane * 16;
@@ -422,6 +430,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               sb[g] = mid ? w[g + 2] : w[g];
             else
               sb[g] = w[g];
+          }
+          if (!slot_free()) {
+            fault = kFaultMmaWait;
+            break;
           }
           tmem_st_32x32b_x4(t_quarter + C::kSfaCol + static_cast<uint32_t>(slot) * C::kSfaSlotCols, a);
 #pragma unroll
@@ -454,6 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               else
                 sb[kb * C::kSfbGroups + g] = w[g];
             }
+          }
+          if (!slot_free()) {
+            fault = kFaultMmaWait;
+            break;
           }
           tmem_st_32x32b_x16(t_quarter + C::kSfaCol + static_cast<uint32_t>(slot) * C::kSfaSlotCols, sa);
 #pragma unroll
