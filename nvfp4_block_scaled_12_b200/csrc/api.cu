@@ -176,7 +176,8 @@ bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
 // (MXFP8) or, with row, one fp32 scale per row passed as sfa / sfb.
 nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
                          int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, GemmTensorMaps* maps,
-                         GemmConfig* cfg, const DeviceInfo** dev, bool mx = false, bool row = false) {
+                         GemmConfig* cfg, const DeviceInfo** dev, bool mx = false, bool row = false,
+                         bool fused = false) {
   if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
   if (M < 1 || M > INT32_MAX / 2) return fail(NVFP4_EINVAL, "M=%lld out of range", (long long)M);
   if (N < 8 || N % 8 != 0 || N > INT32_MAX / 2)
@@ -189,7 +190,7 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   nvfp4_status st = current_device(dev);
   if (st != NVFP4_OK) return st;
 
-  *cfg = gemm_config(M, N);
+  *cfg = gemm_config(M, N, !mx && !row && !fused, (*dev)->num_sms);
   const int bn = cfg->tile_n;
   const int cg = cfg->cta_group;
   *p = GemmParams{};
@@ -528,7 +529,7 @@ nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_
   GemmTensorMaps maps;
   GemmConfig cg;
   const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev);
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev, false, false, true);
   if (st != NVFP4_OK) return st;
   if (any_bf16) {
     st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, ldy, M, ldy * 2, 32, 32,

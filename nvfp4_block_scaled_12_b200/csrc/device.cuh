@@ -555,4 +555,12 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
   for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// Same for a register array filled by several tcgen05.ld.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait_n(uint32_t (&r)[N]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 }  // namespace nvfp4

@@ -48,8 +48,7 @@ namespace {
 
 constexpr int kBKBytes = 128;   // per row per stage: 256 fp4 or 128 fp8 elements
 constexpr uint32_t kABytes = 128 * kBKBytes;  // 16 KB: this CTA's 128 rows of A
-constexpr int kThreads = 352;
-constexpr int kProducers = 2;  // warps 0 and 10
+constexpr int kProducers = 2;
 constexpr uint32_t kTmemCols = 512;
 
 // kCG: CTAs per tile; kBN: tile width; kAcc: accumulator buffers in TMEM;
@@ -58,6 +57,14 @@ constexpr uint32_t kTmemCols = 512;
 // B, applied in the epilogue), otherwise one E8M0 scale per 32 elements.
 template <int kCG, int kBN, int kAcc, bool kMx, bool kRow = false>
 struct Cfg {
+  // Wide tiles (256 columns, one accumulator): the accumulator is drained into
+  // the registers of eight epilogue warps, so the next tile's MMAs can start
+  // before the epilogue's arithmetic and stores.  Other shapes keep four
+  // epilogue warps that read the accumulator chunk by chunk while the MMAs
+  // fill the other buffer.
+  static constexpr bool kWide = kBN == 256 && kAcc == 1;
+  static constexpr int kEpiWarps = kWide ? 8 : 4;
+  static constexpr int kThreads = kWide ? 512 : 352;
   // 512-byte scale atoms (128 rows x 4 scale columns) per 128-row block and
   // k-tile: NVFP4's k-tile is 4 MMA k-blocks of 64 elements with one 4-scale
   // word per row each; MXFP8's is 4 k-blocks of 32 whose scales share one word.
@@ -70,11 +77,15 @@ struct Cfg {
   static constexpr int kSfbBlocks = kBN % 128 == 0 ? kBN / 128 : kBN / 128 + 1;
   static constexpr uint32_t kSfbBytes = kRow ? 0 : kSfbBlocks * kAtoms * 512;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kStagesFit = (224 * 1024 - 4 * 2 * 2048) / kStageBytes;
-  // a multiple of the producer count: each stage then has a single producer
-  // (an mbarrier wait only tells phases apart by parity, so one waiter must
-  // see a stage's phases in order)
-  static constexpr int kStages = (kStagesFit > 8 ? 8 : kStagesFit) / kProducers * kProducers;
+  static constexpr uint32_t kEpiBytes = kEpiWarps * 2 * 2048;  // double-buffered 32 x 32 bf16 staging per warp
+  static constexpr uint32_t kBiasBytes = kWide ? kEpiWarps * 256 : 0;  // each wide epilogue warp's 128 bias values
+  static constexpr int kStagesFit = (224 * 1024 - kEpiBytes - kBiasBytes) / kStageBytes;
+  // The producers alternate k-tiles.  An mbarrier wait tells phases apart
+  // only by parity, so a waiter must never be two phases behind: a producer
+  // has seen the commit of its own previous k-tile (kProducers back), hence
+  // of every k-tile before it, which covers the stage's previous phase as
+  // long as kStages >= kProducers.
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   // TMEM: accumulators, then the scale slots.  Slot j % kSfSlots holds the
   // scales of k-tile j; the movers refill it once the commit of k-tile
   // j - kSfSlots has arrived on that k-tile's empty barrier, which can only
@@ -90,8 +101,9 @@ struct Cfg {
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
   static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
   static constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
-  static constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;  // 4 warps x 2 x 2 KB
-  static constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * 2048;
+  static constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;
+  static constexpr uint32_t kOffBias = kOffEpi + kEpiBytes;
+  static constexpr uint32_t kOffBar = kOffBias + kBiasBytes;
   // full, empty, sfin per stage; acc_full, acc_empty per accumulator; drain
   static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAcc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -102,7 +114,8 @@ struct Cfg {
   static_assert(kSfSlots >= 2 && kSfSlots <= kStages, "TMEM budget");
   static_assert(kSfaCol % kSfaSlotCols == 0 && kSfbCol % 8 == 0 && kSfbSlotCols % 8 == 0, "tcgen05.st column alignment");
   static_assert(kSfbCol + kSfSlots * kSfbSlotCols <= kTmemCols, "TMEM budget");
-  static_assert(kStages >= 3, "pipeline depth");
+  static_assert(kStages >= 3 && kStages >= kProducers, "pipeline depth");
+  static_assert(!kWide || (kCG == 2 && !kMx), "wide tiles are NVFP4 CTA pairs");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -135,13 +148,14 @@ __device__ __forceinline__ void store_chunk_bf16(const CUtensorMap* tmap, uint8_
 }
 
 template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ GemmParams p) {
   using C = Cfg<kCG, kBN, kAcc, kMx, kRow>;
   static_assert(!(kFused && kMx), "the fused quantize epilogue writes NVFP4 after an NVFP4 GEMM");
   static_assert(!kRow || kMx, "row-wise FP8 uses the 8-bit operand layout");
+  static_assert(!(C::kWide && kFused), "the fused epilogue uses the double-buffered tile shapes");
   constexpr int S = C::kStages;
   constexpr int R = C::kSfSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -160,6 +174,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = kCG == 2 ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
+  // Warp roles.  Standard layout (11 warps): 0 and 10 TMA producers, 1 MMA,
+  // 2-5 epilogue, 6-9 scale movers.  Wide layout (16 warps, four warpgroups):
+  // 0 and 2 producers, 1 MMA, 3 idle, 4-11 epilogue (two per TMEM lane
+  // quarter, one per 128-column half), 12-15 scale movers.
+  const bool is_producer = C::kWide ? (warp == 0 || warp == 2) : (warp == 0 || warp == 10);
+  const bool is_mover = C::kWide ? warp >= 12 : (warp >= 6 && warp <= 9);
+  const bool is_epilogue = C::kWide ? (warp >= 4 && warp < 12) : (warp >= 2 && warp <= 5);
   const int cluster = blockIdx.x / kCG;
   const int num_clusters = gridDim.x / kCG;
 
@@ -172,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < kAcc; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4 * kCG);
+      mbar_init(&acc_empty[a], C::kEpiWarps * kCG);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -213,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(bar);
   };
 
-  if (warp == 0 || warp == 10) {
+  auto run_producer = [&]() {
     // ------------------------------------------------------------ producers
     if (lane == 0) {
       const int pid = warp == 0 ? 0 : 1;
@@ -276,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  };
+  auto run_mma = [&]() {
     // ------------------------------------------------------------ MMA issuer (group leader)
     if (lane == 0 && leader) {
       // one MMA k-block: NVFP4 reads 4 scale columns per k-block; MXFP8 reads
@@ -366,10 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(drain, 0u, nullptr)) fault |= kFaultDrainWait;
     }
     __syncwarp();
-  } else if (warp >= 6 && kRow) {
-    // row-wise FP8 has no block scales to move
-  } else if (warp >= 6) {
-    // ------------------------------------------------------------ scale movers (warps 6-9)
+  };
+  auto run_movers = [&]() {
+    // ------------------------------------------------------------ scale movers
     const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter of this warp
     const uint32_t t_quarter = tmem_base + ((q * 32u) << 16);
     int stage = 0;
@@ -489,7 +510,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (fault != 0u) *abort_flag = 1;
-  } else {
+  };
+  auto run_epilogue_wide = [&]() {
+    if constexpr (C::kWide) {
+    // ------------------------------------------------------------ epilogue, wide tiles
+    // Warp e (0-7) owns TMEM lane quarter e % 4 (rows 32q..32q+31 of this
+    // CTA's 128) and columns 128h..128h+127 of the tile, h = e / 4.  It reads
+    // its whole slice into registers, hands the accumulator back at once, and
+    // only then applies alpha and bias and stores bf16 through the TMA.
+    const int e = warp - 4;
+    const int q = warp & 3;
+    const int h = e >> 2;
+    uint8_t* stage_buf = smem + C::kOffEpi + e * 4096;
+    uint8_t* bias_buf = smem + C::kOffBias + e * 256;
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    const float alpha = p.alpha_scale != nullptr ? __fmul_rn(p.alpha, *p.alpha_scale) : p.alpha;
+    for (int tile = cluster; tile < p.num_tiles; tile += num_clusters) {
+      const int tm = tile % p.tiles_m;
+      const int c0 = (tile / p.tiles_m) * kBN + h * 128;  // first column of this warp's slice
+      // this slice's bias (4 values per lane), staged while the MMAs run
+      __syncwarp();  // every lane is done with the previous tile's values
+      {
+        uint2 bv = make_uint2(0u, 0u);
+        const int cb = c0 + lane * 4;
+        if (p.bias != nullptr && cb < p.N) bv = __ldg(reinterpret_cast<const uint2*>(p.bias + cb));
+        *reinterpret_cast<uint2*>(bias_buf + lane * 8) = bv;
+      }
+      const bool got = mbar_wait(&acc_full[0], acc_phase, abort_flag);
+      __syncwarp();  // tcgen05.ld below needs the whole warp converged
+      if (!__all_sync(0xffffffffu, got)) {
+        fault = kFaultEpilogueWait;
+        break;
+      }
+      tc_fence_after();
+      const int row_base = (tm * kCG + static_cast<int>(rank)) * 128 + q * 32;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128);
+      uint32_t r[128];
+      tmem_ld_32x32b_x32(t_row + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+      tmem_ld_32x32b_x32(t_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      tmem_ld_32x32b_x32(t_row + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+      tmem_ld_32x32b_x32(t_row + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+      tmem_ld_wait_n<128>(r);
+      // the accumulator is in registers: the next tile's MMAs may start
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_leader(&acc_empty[0]);
+      acc_phase ^= 1u;
+      if (row_base < p.M) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int n = c0 + c * 32;
+          if (n < p.N) {
+            uint32_t w[16];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint4 b = *reinterpret_cast<const uint4*>(bias_buf + c * 64 + g * 16);
+              const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int j = c * 32 + g * 8 + 2 * t;
+                w[4 * g + t] = pack_bf16x2(fmaf(alpha, __uint_as_float(r[j]), bf16_lo(bw[t])),
+                                           fmaf(alpha, __uint_as_float(r[j + 1]), bf16_hi(bw[t])));
+              }
+            }
+            store_chunk_bf16(&tmap_y, stage_buf + buf * 2048, w, lane, n, row_base);
+            buf ^= 1;
+          }
+        }
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+    if (fault != 0u) *abort_flag = 1;
+    }
+  };
+  auto run_epilogue = [&]() {
+    if constexpr (!C::kWide) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     uint8_t* stage_buf = smem + C::kOffEpi + (warp - 2) * 4096;
@@ -615,6 +711,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) bulk_wait<0>();
     if (fault != 0u) *abort_flag = 1;
+    }
+  };
+
+  if constexpr (C::kWide) {
+    // One role per warpgroup, each with its own register budget (512 threads
+    // x 128 at launch): the two epilogue warpgroups hold a 128-column
+    // accumulator slice per thread; 56 + 88 + 2 x 184 = 4 x 128.
+    const int wg = warp >> 2;
+    if (wg == 0) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+      if (warp == 0 || warp == 2)
+        run_producer();
+      else if (warp == 1)
+        run_mma();
+    } else if (wg == 3) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+      run_movers();
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
+      run_epilogue_wide();
+    }
+  } else {
+    if (is_producer)
+      run_producer();
+    else if (warp == 1)
+      run_mma();
+    else if (is_mover) {
+      if constexpr (!kRow) run_movers();  // row-wise FP8 has no block scales to move
+    } else if (is_epilogue)
+      run_epilogue();
   }
 
   if (fault != 0u && lane == 0 && p.fault != nullptr) atomicOr(p.fault, fault);
@@ -635,7 +761,7 @@ cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t st
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -666,10 +792,14 @@ cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t st
 
 }  // namespace
 
-GemmConfig gemm_config(int64_t M, int64_t N) {
-  (void)N;
-  if (M > 128) return GemmConfig{2, 192, 2};
-  return GemmConfig{1, 192, 2};
+GemmConfig gemm_config(int64_t M, int64_t N, bool plain_nvfp4, int num_sms) {
+  if (M <= 128) return GemmConfig{1, 192, 2};
+  // 256 x 256 tiles do a third more MMA work per pipeline step than 256 x 192
+  // ones for the same per-k-tile synchronisation, but leave SMs idle when
+  // there are fewer tiles than CTA pairs.
+  const int64_t wide_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  if (plain_nvfp4 && wide_tiles >= num_sms / 2) return GemmConfig{2, 256, 1};
+  return GemmConfig{2, 192, 2};
 }
 
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
@@ -694,10 +824,9 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
                  : launch<CG, BN, ACC, false, false>(m, p, stream, dev);
   NVFP4_GEMM_CASE(2, 192, 2)
   NVFP4_GEMM_CASE(1, 192, 2)
-  NVFP4_GEMM_CASE(2, 128, 2)
-  NVFP4_GEMM_CASE(1, 128, 2)
-  NVFP4_GEMM_CASE(2, 256, 1)
 #undef NVFP4_GEMM_CASE
+  if (c.cta_group == 2 && c.tile_n == 256 && c.acc_bufs == 1 && !fused)
+    return launch<2, 256, 1, false, false>(m, p, stream, dev);
   return cudaErrorInvalidConfiguration;
 }
 

@@ -160,5 +160,79 @@ def test_gemm_is_deterministic(F):
     assert torch.equal(y1, y2)
 
 
+def _wide(M, N):
+    """True when the library takes its 256 x 256 CTA-pair tiles for this
+    plain NVFP4 GEMM: at least one tile per CTA pair of the device."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return ((M + 255) // 256) * ((N + 255) // 256) >= sms // 2
+
+
+@pytest.mark.parametrize("m,n,k", [(2341, 2056, 3136), (4608, 3072, 3072), (2305, 8200, 1088)])
+def test_wide_tiles_ragged_sampled(F, m, n, k):
+    # Shapes that take the 256 x 256 tiles, ragged in M, N and K (a last
+    # k-tile with one or two MMA k-blocks): all columns of sampled rows (the
+    # last rows included) and all rows of sampled columns (the last included).
+    assert _wide(m, n)
+    wl = synth.LinearWorkload(f"wide_{m}x{n}x{k}", m, k, n, seed=m + 3 * n + k)
+    rng = np.random.default_rng(m + n)
+    rows = np.unique(np.r_[rng.choice(m, 64, replace=False), m - 1, m - 2, 255, 256])
+    y = _check_linear(F, wl, rows=rows)
+    x, w, b = wl.activations(), wl.weight(), wl.bias_vec()
+    (xc, xs, gx), (wc, ws, gw) = _oracle_layer(x, w)
+    cols = np.unique(np.r_[rng.choice(n, 64, replace=False), n - 1, n - 8, 127, 128, 255, 256])
+    y_ref = O.gemm_ref(xc, xs, gx, wc[cols], ws[cols], gw, b.float().numpy()[cols])
+    tol = O.gemm_tolerance(xc, xs, gx, wc[cols], ws[cols], gw, y_ref)
+    assert_within_tol(y[:, cols], y_ref, tol, wl.name + " columns")
+
+
+@pytest.mark.parametrize("side", ["a", "b"])
+@pytest.mark.parametrize("row,kblk", [(0, 0), (131, 3), (255, 17), (256, 6), (700, 31), (2303, 9)])
+def test_wide_tiles_scale_layout_probe(F, side, row, kblk):
+    # As test_scale_layout_probe, on a shape that takes the 256 x 256 tiles:
+    # the probed row lands in either 128-row half of an A tile and in either
+    # 128-column half of a B tile.
+    M = N = 2304
+    K = 512
+    assert _wide(M, N)
+    ac, asf = _uniform_operand(M, K)
+    bc, bsf = _uniform_operand(N, K)
+    (asf if side == "a" else bsf)[row, kblk] = 0x40  # 2.0
+    y = _run_raw(F, ac, asf, bc, bsf)
+    want = np.full((M, N), float(K))
+    if side == "a":
+        want[row, :] += 16
+    else:
+        want[:, row] += 16
+    bad = np.argwhere(y != want)
+    assert bad.size == 0, f"{bad.shape[0]} wrong, first {bad[:4].tolist()} got {y[tuple(bad[0])]}"
+
+
+def test_wide_tiles_exact_accumulation_is_bit_exact(F):
+    rng = np.random.default_rng(21)
+    M, N, K = 2304, 2304, 256
+    assert _wide(M, N)
+    a_codes = rng.integers(0, 256, (M, K // 2)).astype(np.uint8)
+    b_codes = rng.integers(0, 256, (N, K // 2)).astype(np.uint8)
+    pow2 = np.array([0x30, 0x38, 0x40], np.uint8)
+    a_sf = rng.choice(pow2, (M, K // 16))
+    b_sf = rng.choice(pow2, (N, K // 16))
+    bias = O.round_to_bf16(rng.integers(-64, 64, N) * 0.5)
+    y = _run_raw(F, a_codes, a_sf, b_codes, b_sf, alpha=0.5, bias=bias.astype(np.float32))
+    want = O.round_to_bf16(O.gemm_ref(a_codes, a_sf, 1.0, b_codes, b_sf, 1.0, None) * 0.5 + bias)
+    bad = np.argwhere(y != want)
+    assert bad.size == 0, f"{bad.shape[0]} differ, first {bad[:4].tolist()}: {y[tuple(bad[0])]} vs {want[tuple(bad[0])]}"
+
+
+def test_wide_tiles_are_deterministic(F):
+    wl = synth.LinearWorkload("det_wide", 4608, 1024, 4096, seed=10)
+    assert _wide(wl.m, wl.n)
+    xq, wq = _gpu_layer(F, wl.activations(), wl.weight())
+    b = wl.bias_vec().cuda()
+    y1 = F.gemm(xq, wq, bias=b)
+    y2 = F.gemm(xq, wq, bias=b)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
 def test_no_kernel_reported_a_fault(F):
     F.nvfp4_check_fault()
