@@ -209,14 +209,6 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   p->alpha = alpha;
   p->bias = static_cast<const __nv_bfloat16*>(bias);
   p->fault = (*dev)->fault;
-  p->pf_ptr[0] = b;  // weights first: every tile of a wave touches new weight rows
-  p->pf_bytes[0] = static_cast<uint64_t>(N) * static_cast<uint64_t>(row_bytes);
-  p->pf_ptr[1] = a;
-  p->pf_bytes[1] = static_cast<uint64_t>(M) * static_cast<uint64_t>(row_bytes);
-  p->pf_ptr[2] = sfb;
-  p->pf_bytes[2] = row ? static_cast<uint64_t>(N) * 4 : mx ? nvfp4_mxfp8_sf_bytes(N, K) : nvfp4_sf_bytes(N, K);
-  p->pf_ptr[3] = sfa;
-  p->pf_bytes[3] = row ? static_cast<uint64_t>(M) * 4 : mx ? nvfp4_mxfp8_sf_bytes(M, K) : nvfp4_sf_bytes(M, K);
 
   st = make_tmap(&maps->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, row_bytes, M, row_bytes, 128, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B, "A");

@@ -4,13 +4,19 @@
 // epilogue and an optional fused epilogue that quantizes the result for the
 // next layer.
 //
-// One persistent kernel, templated on the CTA-group size kCG:
-//   kCG = 2  a CTA pair (cluster of 2) owns a 256 x 192 output tile: each
-//            CTA loads its 128 rows of A and its 96 rows of B, and the pair
-//            leader issues tcgen05.mma.cta_group::2 (M=256, N=192, K=64), so
-//            every B byte crosses L2 once per pair.  Used for M > 128.
-//   kCG = 1  one CTA owns a 128 x 192 tile (small M).
-// Warps (11 per CTA):
+// One persistent kernel, templated on the tile shape:
+//   256 x 256 (wide)  a CTA pair (cluster of 2) owns the tile: each CTA loads
+//            its 128 rows of A and 128 rows of B, and the pair leader issues
+//            tcgen05.mma.cta_group::2 (M=256, N=256, K=64) into one
+//            256-column accumulator.  Used for plain NVFP4 GEMMs with at
+//            least one tile per CTA pair.
+//   256 x 192  a CTA pair with 96 rows of B per CTA and two accumulators
+//            (M > 128 otherwise, MXFP8, row-wise FP8, the fused epilogue).
+//   128 x 192  one CTA per tile (M <= 128).
+// Every pipeline step (one 128-byte k-tile: four MMAs) costs the MMA-issuing
+// thread a barrier wait, a commit and its bookkeeping, during which the
+// tensor pipe runs dry; the wide tile does a third more MMA work per step.
+// Warps, standard layout (11 per CTA):
 //   0, 10 TMA producers, alternating k-tiles: A/B tiles (128-byte rows,
 //         128-byte swizzle) and the scale atoms (3-D boxes, zero-filled past
 //         K and past the last row block) into a shared-memory ring.  A TMA
@@ -18,9 +24,8 @@
 //         cannot keep the SM's TMA unit busy; two issuing warps reach about
 //         twice the load rate.
 //   1     allocates TMEM; in the leader one thread waits for one barrier per
-//         k-tile, issues the MMAs into a double-buffered fp32 accumulator and
-//         commits once: that commit frees the shared-memory stage and the
-//         TMEM scale slot of the k-tile together.
+//         k-tile, issues the MMAs and commits once: that commit frees the
+//         shared-memory stage and the TMEM scale slot of the k-tile together.
 //   2-5   epilogue: tcgen05.ld 32 columns at a time, alpha*acc + bias, bf16,
 //         swizzled staging in shared memory, TMA store (or the fused
 //         quantize); drains accumulator i while the MMA fills i^1.
@@ -31,6 +36,10 @@
 //         a full copy.  Register-path stores run beside the tensor pipe, where
 //         tcgen05.cp copies of the same (replicated) data would serialize with
 //         the MMAs.
+// Wide layout (16 warps = four warpgroups with their own register budgets):
+//   0, 2 producers, 1 MMA issuer, 3 idle; 4-11 epilogue, two warps per lane
+//   quarter (one per 128-column half), each reading its whole 128-column
+//   slice into registers before releasing the accumulator; 12-15 movers.
 // TMEM columns: the accumulators first, then the scale slots: 16 columns of A
 // scales each (4 per MMA k-block), then kBN/8 columns of B scales each
 // (kBN/32 per k-block).  Scale column j of lane l holds the 4 scales of row
@@ -238,20 +247,6 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     // ------------------------------------------------------------ producers
     if (lane == 0) {
       const int pid = warp == 0 ? 0 : 1;
-      if (pid == 0) {
-        // Every CTA first asks L2 for its 1/gridDim share of the operands: all
-        // of them fit in L2, and a stage whose rows include one first touch
-        // would otherwise wait the full DRAM latency.
-        for (int i = 0; i < 4; ++i) {
-          const uint64_t share = ((p.pf_bytes[i] + gridDim.x - 1) / gridDim.x + 15) & ~uint64_t(15);
-          const uint64_t begin = share * blockIdx.x;
-          const uint64_t end = begin + share < p.pf_bytes[i] ? begin + share : p.pf_bytes[i];
-          for (uint64_t off = begin; off < end; off += 65536) {
-            const uint64_t n = end - off < 65536 ? end - off : 65536;
-            prefetch_l2_bulk(p.pf_ptr[i] + off, static_cast<uint32_t>(n));
-          }
-        }
-      }
       // flattened (tile, k-tile) sequence of this CTA group; producer pid
       // issues the entries j with j % kProducers == pid into stage j % S
       const int my_tiles = p.num_tiles > cluster ? (p.num_tiles - cluster + num_clusters - 1) / num_clusters : 0;

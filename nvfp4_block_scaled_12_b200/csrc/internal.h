@@ -34,9 +34,6 @@ struct GemmParams {
   const float* col_scale;     // row-wise FP8: [N] scales of B's rows (output columns)
   const __nv_bfloat16* bias;  // nullable
   unsigned* fault;
-  // operand byte ranges prefetched into L2 at kernel start (A, B, SFA, SFB)
-  const uint8_t* pf_ptr[4];
-  uint64_t pf_bytes[4];
   // fused epilogue (only read by the fused kernel)
   int32_t n_ranges;
   EpiRange ranges[NVFP4_MAX_RANGES];
