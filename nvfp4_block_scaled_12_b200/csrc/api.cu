@@ -190,7 +190,7 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   nvfp4_status st = current_device(dev);
   if (st != NVFP4_OK) return st;
 
-  *cfg = gemm_config(M, N, !mx && !row && !fused, (*dev)->num_sms);
+  *cfg = gemm_config(M, N, (*dev)->num_sms);
   const int bn = cfg->tile_n;
   const int cg = cfg->cta_group;
   *p = GemmParams{};

@@ -124,7 +124,7 @@ struct Cfg {
   static_assert(kSfaCol % kSfaSlotCols == 0 && kSfbCol % 8 == 0 && kSfbSlotCols % 8 == 0, "tcgen05.st column alignment");
   static_assert(kSfbCol + kSfSlots * kSfbSlotCols <= kTmemCols, "TMEM budget");
   static_assert(kStages >= 3 && kStages >= kProducers, "pipeline depth");
-  static_assert(!kWide || (kCG == 2 && !kMx), "wide tiles are NVFP4 CTA pairs");
+  static_assert(!kWide || kCG == 2, "wide tiles are CTA pairs");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -164,7 +164,6 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
   using C = Cfg<kCG, kBN, kAcc, kMx, kRow>;
   static_assert(!(kFused && kMx), "the fused quantize epilogue writes NVFP4 after an NVFP4 GEMM");
   static_assert(!kRow || kMx, "row-wise FP8 uses the 8-bit operand layout");
-  static_assert(!(C::kWide && kFused), "the fused epilogue uses the double-buffered tile shapes");
   constexpr int S = C::kStages;
   constexpr int R = C::kSfSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -506,6 +505,65 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     }
     if (fault != 0u) *abort_flag = 1;
   };
+  // One 32-column chunk of a 32-row slice, as bf16 words (w[j] = columns 2j,
+  // 2j+1 of this thread's row): the fused epilogue's column ranges pick the
+  // destination and activation; bf16 chunks go out through the TMA, NVFP4
+  // chunks are quantized (two 16-element blocks) into the next layer's codes
+  // and swizzled scales (sf_word collects the 64-column group's scale word).
+  const int m_padded = (p.M + 127) & ~127;  // rows of the next layer's scale buffer
+  auto emit_chunk = [&](uint32_t (&w)[16], int n, int row_base, uint8_t* stage_buf, int& buf, uint32_t& sf_word) {
+    const int row = row_base + lane;
+    int act = NVFP4_ACT_NONE, dst = NVFP4_DST_BF16, out_col = n;
+    if (kFused) {
+      int hit = -1;
+      for (int i = 0; i < p.n_ranges; ++i)
+        if (n >= p.ranges[i].begin && n < p.ranges[i].end) hit = i;
+      if (hit < 0) return;
+      act = p.ranges[hit].act;
+      dst = p.ranges[hit].dst;
+      out_col = p.ranges[hit].dst_col + (n - p.ranges[hit].begin);
+    }
+    if (kFused && act == NVFP4_ACT_GELU_TANH) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        w[j] = pack_bf16x2(gelu_tanh_f32(bf16_lo(w[j])), gelu_tanh_f32(bf16_hi(w[j])));
+    }
+    if (!kFused || dst == NVFP4_DST_BF16) {
+      if (row_base < p.M) {
+        store_chunk_bf16(&tmap_y, stage_buf + buf * 2048, w, lane, out_col, row_base);
+        buf ^= 1;
+      }
+    } else {
+      // next layer's NVFP4 input: two 16-element blocks per chunk
+      const float g = p.g_next;
+      const float d6 = __fmul_rn(6.0f, g);
+      float blk[16];
+      uint32_t c0, c1, c2, c3;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        blk[2 * j] = bf16_lo(w[j]);
+        blk[2 * j + 1] = bf16_hi(w[j]);
+      }
+      const uint32_t s0 = quantize_block16(blk, g, d6, c0, c1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        blk[2 * j] = bf16_lo(w[8 + j]);
+        blk[2 * j + 1] = bf16_hi(w[8 + j]);
+      }
+      const uint32_t s1 = quantize_block16(blk, g, d6, c2, c3);
+      if (row < p.M)
+        *reinterpret_cast<uint4*>(p.codes_next + static_cast<size_t>(row) * (p.k_next >> 1) + (out_col >> 1)) =
+            make_uint4(c0, c1, c2, c3);
+      const int csf = out_col >> 4;  // scale column of the first block (even)
+      sf_word |= (s0 | (s1 << 8)) << (8 * (csf & 3));
+      if ((csf & 3) == 2) {  // the 64-column group is complete
+        const uint32_t word = row < p.M ? sf_word : 0u;  // padding rows of the scale buffer are zero
+        if (row < m_padded) *reinterpret_cast<uint32_t*>(p.sf_next + sf_offset(row, csf & ~3, p.k_next >> 6)) = word;
+        sf_word = 0u;
+      }
+    }
+  };
+
   auto run_epilogue_wide = [&]() {
     if constexpr (C::kWide) {
     // ------------------------------------------------------------ epilogue, wide tiles
@@ -552,27 +610,38 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
       __syncwarp();
       if (lane == 0) arrive_leader(&acc_empty[0]);
       acc_phase ^= 1u;
-      if (row_base < p.M) {
+      // y = bf16(alpha * acc + bias) (row-wise FP8: fl(s_a[row] * s_b[n]) in
+      // place of alpha), packed two columns per word
+      const int row = row_base + lane;
+      const float sa = kRow ? (row < p.M ? __ldg(p.row_scale + row) : 0.0f) : 0.0f;
+      uint32_t sf_word = 0u;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int n = c0 + c * 32;
-          if (n < p.N) {
-            uint32_t w[16];
+      for (int c = 0; c < 4; ++c) {
+        const int n = c0 + c * 32;
+        if (n >= p.N) break;
+        uint32_t w[16];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint4 b = *reinterpret_cast<const uint4*>(bias_buf + c * 64 + g * 16);
-              const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const int j = c * 32 + g * 8 + 2 * t;
-                w[4 * g + t] = pack_bf16x2(fmaf(alpha, __uint_as_float(r[j]), bf16_lo(bw[t])),
-                                           fmaf(alpha, __uint_as_float(r[j + 1]), bf16_hi(bw[t])));
-              }
+        for (int g = 0; g < 4; ++g) {
+          const uint4 b = *reinterpret_cast<const uint4*>(bias_buf + c * 64 + g * 16);
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+          float4 cs0 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), cs1 = cs0;
+          if constexpr (kRow) {
+            if (n + 8 * g < p.N) {
+              cs0 = __ldg(reinterpret_cast<const float4*>(p.col_scale + n + 8 * g));
+              cs1 = __ldg(reinterpret_cast<const float4*>(p.col_scale + n + 8 * g + 4));
             }
-            store_chunk_bf16(&tmap_y, stage_buf + buf * 2048, w, lane, n, row_base);
-            buf ^= 1;
+          }
+          const float csv[8] = {cs0.x, cs0.y, cs0.z, cs0.w, cs1.x, cs1.y, cs1.z, cs1.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int j = c * 32 + g * 8 + 2 * t;
+            const float a0 = kRow ? __fmul_rn(sa, csv[2 * t]) : alpha;
+            const float a1 = kRow ? __fmul_rn(sa, csv[2 * t + 1]) : alpha;
+            w[4 * g + t] = pack_bf16x2(fmaf(a0, __uint_as_float(r[j]), bf16_lo(bw[t])),
+                                       fmaf(a1, __uint_as_float(r[j + 1]), bf16_hi(bw[t])));
           }
         }
+        emit_chunk(w, n, row_base, stage_buf, buf, sf_word);
       }
     }
     if (lane == 0) bulk_wait<0>();
@@ -587,7 +656,6 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    const int m_padded = (p.M + 127) & ~127;  // rows of the next layer's scale buffer
     // alpha = g_a * g_b; with a scale measured on the device, g_a is read here
     const float alpha = p.alpha_scale != nullptr ? __fmul_rn(p.alpha, *p.alpha_scale) : p.alpha;
     for (int tile = cluster; tile < p.num_tiles; tile += num_clusters) {
@@ -617,87 +685,39 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
         }
         const int n = n0 + c * 32;
         if (n >= p.N) continue;
-
-        // which output, and which activation, this chunk goes to
-        int act = NVFP4_ACT_NONE, dst = NVFP4_DST_BF16, out_col = n;
-        if (kFused) {
-          int hit = -1;
-          for (int i = 0; i < p.n_ranges; ++i)
-            if (n >= p.ranges[i].begin && n < p.ranges[i].end) hit = i;
-          if (hit < 0) continue;
-          act = p.ranges[hit].act;
-          dst = p.ranges[hit].dst;
-          out_col = p.ranges[hit].dst_col + (n - p.ranges[hit].begin);
+        if (kFused) {  // chunks outside every column range are not written
+          bool hit = false;
+          for (int i = 0; i < p.n_ranges; ++i) hit |= n >= p.ranges[i].begin && n < p.ranges[i].end;
+          if (!hit) continue;
         }
-
-        float bias[32];
+        uint32_t w[16];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           uint4 b = make_uint4(0u, 0u, 0u, 0u);
           if (p.bias != nullptr && n + 8 * g < p.N) b = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8 * g));
-          bias[8 * g + 0] = bf16_lo(b.x);
-          bias[8 * g + 1] = bf16_hi(b.x);
-          bias[8 * g + 2] = bf16_lo(b.y);
-          bias[8 * g + 3] = bf16_hi(b.y);
-          bias[8 * g + 4] = bf16_lo(b.z);
-          bias[8 * g + 5] = bf16_hi(b.z);
-          bias[8 * g + 6] = bf16_lo(b.w);
-          bias[8 * g + 7] = bf16_hi(b.w);
-        }
-        float v[32];
-        if constexpr (kRow) {
-          // row-wise FP8: y = fl(s_a[row] * s_b[n]) * acc + bias
-          const float sa = row < p.M ? __ldg(p.row_scale + row) : 0.0f;
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+          if constexpr (kRow) {
+            // row-wise FP8: y = fl(s_a[row] * s_b[n]) * acc + bias
+            const float sa = row < p.M ? __ldg(p.row_scale + row) : 0.0f;
+            float4 cs0 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), cs1 = cs0;
+            if (n + 8 * g < p.N) {
+              cs0 = __ldg(reinterpret_cast<const float4*>(p.col_scale + n + 8 * g));
+              cs1 = __ldg(reinterpret_cast<const float4*>(p.col_scale + n + 8 * g + 4));
+            }
+            const float csv[8] = {cs0.x, cs0.y, cs0.z, cs0.w, cs1.x, cs1.y, cs1.z, cs1.w};
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            float4 cs = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (n + 4 * g < p.N) cs = __ldg(reinterpret_cast<const float4*>(p.col_scale + n + 4 * g));
-            v[4 * g + 0] = round_bf16(fmaf(__fmul_rn(sa, cs.x), __uint_as_float(r[4 * g + 0]), bias[4 * g + 0]));
-            v[4 * g + 1] = round_bf16(fmaf(__fmul_rn(sa, cs.y), __uint_as_float(r[4 * g + 1]), bias[4 * g + 1]));
-            v[4 * g + 2] = round_bf16(fmaf(__fmul_rn(sa, cs.z), __uint_as_float(r[4 * g + 2]), bias[4 * g + 2]));
-            v[4 * g + 3] = round_bf16(fmaf(__fmul_rn(sa, cs.w), __uint_as_float(r[4 * g + 3]), bias[4 * g + 3]));
-          }
-        } else {
+            for (int t = 0; t < 4; ++t)
+              w[4 * g + t] = pack_bf16x2(fmaf(__fmul_rn(sa, csv[2 * t]), __uint_as_float(r[8 * g + 2 * t]), bf16_lo(bw[t])),
+                                         fmaf(__fmul_rn(sa, csv[2 * t + 1]), __uint_as_float(r[8 * g + 2 * t + 1]),
+                                              bf16_hi(bw[t])));
+          } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = round_bf16(fmaf(alpha, __uint_as_float(r[j]), bias[j]));
-        }
-        if (kFused && act == NVFP4_ACT_GELU_TANH) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = round_bf16(gelu_tanh_f32(v[j]));
-        }
-
-        if (!kFused || dst == NVFP4_DST_BF16) {
-          if (row_base < p.M) {
-            uint32_t w[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-            store_chunk_bf16(&tmap_y, stage_buf + buf * 2048, w, lane, out_col, row_base);
-            buf ^= 1;
-          }
-        } else {
-          // next layer's NVFP4 input: two 16-element blocks per chunk
-          const float g = p.g_next;
-          const float d6 = __fmul_rn(6.0f, g);
-          float blk[16];
-          uint32_t c0, c1, c2, c3;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) blk[j] = v[j];
-          const uint32_t s0 = quantize_block16(blk, g, d6, c0, c1);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) blk[j] = v[16 + j];
-          const uint32_t s1 = quantize_block16(blk, g, d6, c2, c3);
-          if (row < p.M)
-            *reinterpret_cast<uint4*>(p.codes_next + static_cast<size_t>(row) * (p.k_next >> 1) + (out_col >> 1)) =
-                make_uint4(c0, c1, c2, c3);
-          const int csf = out_col >> 4;  // scale column of the first block (even)
-          sf_word |= (s0 | (s1 << 8)) << (8 * (csf & 3));
-          if ((csf & 3) == 2) {  // the 64-column group is complete
-            const uint32_t word = row < p.M ? sf_word : 0u;  // padding rows of the scale buffer are zero
-            if (row < m_padded)
-              *reinterpret_cast<uint32_t*>(p.sf_next + sf_offset(row, csf & ~3, p.k_next >> 6)) = word;
-            sf_word = 0u;
+            for (int t = 0; t < 4; ++t)
+              w[4 * g + t] = pack_bf16x2(fmaf(alpha, __uint_as_float(r[8 * g + 2 * t]), bf16_lo(bw[t])),
+                                         fmaf(alpha, __uint_as_float(r[8 * g + 2 * t + 1]), bf16_hi(bw[t])));
           }
         }
+        emit_chunk(w, n, row_base, stage_buf, buf, sf_word);
       }
       if (++acc == kAcc) {
         acc = 0;
@@ -722,7 +742,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
         run_mma();
     } else if (wg == 3) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
-      run_movers();
+      if constexpr (!kRow) run_movers();  // row-wise FP8 has no block scales to move
     } else {
       asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
       run_epilogue_wide();
@@ -787,13 +807,13 @@ cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t st
 
 }  // namespace
 
-GemmConfig gemm_config(int64_t M, int64_t N, bool plain_nvfp4, int num_sms) {
+GemmConfig gemm_config(int64_t M, int64_t N, int num_sms) {
   if (M <= 128) return GemmConfig{1, 192, 2};
   // 256 x 256 tiles do a third more MMA work per pipeline step than 256 x 192
   // ones for the same per-k-tile synchronisation, but leave SMs idle when
   // there are fewer tiles than CTA pairs.
   const int64_t wide_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-  if (plain_nvfp4 && wide_tiles >= num_sms / 2) return GemmConfig{2, 256, 1};
+  if (wide_tiles >= num_sms / 2) return GemmConfig{2, 256, 1};
   return GemmConfig{2, 192, 2};
 }
 
@@ -801,6 +821,8 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
                         cudaStream_t stream, const DeviceInfo& dev, bool row) {
   if (row) {  // row-wise FP8: the default tile shapes, no fused epilogue
     if (fused || !mx) return cudaErrorInvalidConfiguration;
+    if (c.cta_group == 2 && c.tile_n == 256 && c.acc_bufs == 1)
+      return launch<2, 256, 1, false, true, true>(m, p, stream, dev);
     if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2)
       return launch<2, 192, 2, false, true, true>(m, p, stream, dev);
     if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2)
@@ -809,6 +831,7 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
   }
   if (mx) {  // MXFP8 operands: the default tile shapes, no fused epilogue
     if (fused) return cudaErrorInvalidConfiguration;
+    if (c.cta_group == 2 && c.tile_n == 256 && c.acc_bufs == 1) return launch<2, 256, 1, false, true>(m, p, stream, dev);
     if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2) return launch<2, 192, 2, false, true>(m, p, stream, dev);
     if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2) return launch<1, 192, 2, false, true>(m, p, stream, dev);
     return cudaErrorInvalidConfiguration;
@@ -817,11 +840,10 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
   if (c.cta_group == CG && c.tile_n == BN && c.acc_bufs == ACC)                                             \
     return fused ? launch<CG, BN, ACC, true, false>(m, p, stream, dev)                                      \
                  : launch<CG, BN, ACC, false, false>(m, p, stream, dev);
+  NVFP4_GEMM_CASE(2, 256, 1)
   NVFP4_GEMM_CASE(2, 192, 2)
   NVFP4_GEMM_CASE(1, 192, 2)
 #undef NVFP4_GEMM_CASE
-  if (c.cta_group == 2 && c.tile_n == 256 && c.acc_bufs == 1 && !fused)
-    return launch<2, 256, 1, false, false>(m, p, stream, dev);
   return cudaErrorInvalidConfiguration;
 }
 

@@ -78,9 +78,7 @@ struct GemmConfig {
   int tile_n;     // output tile width
   int acc_bufs;   // accumulator buffers in TMEM
 };
-// plain_nvfp4: an NVFP4 GEMM with the bf16 epilogue (not MXFP8, row-wise FP8
-// or the fused quantize epilogue), which may use the wide 256 x 256 tiles.
-GemmConfig gemm_config(int64_t M, int64_t N, bool plain_nvfp4, int num_sms);
+GemmConfig gemm_config(int64_t M, int64_t N, int num_sms);
 // mx: MXFP8 operands (E4M3 codes [rows, K], E8M0 scales) instead of NVFP4.
 // row: row-wise FP8 (8-bit operands without block scales; requires mx).
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,

@@ -119,6 +119,16 @@ def test_fused_single_stream_block_shape_sampled(F):
     _check_fused(F, wl, synth.SINGLE_Q, synth.SINGLE_KV, synth.SINGLE_MLP, rows=rows)
 
 
+def test_fused_wide_tiles_ragged_sampled(F):
+    # A shape that takes the 256 x 256 tiles (at least one per CTA pair), ragged
+    # in M and with range boundaries inside tiles and inside 128-column halves.
+    wl = synth.LinearWorkload("fused_wide", 2341, 1088, 8288, seed=23)  # columns 8256.. in no range
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert ((wl.m + 255) // 256) * ((wl.n + 255) // 256) >= sms // 2
+    rows = np.unique(np.r_[np.random.default_rng(23).choice(wl.m, 40, replace=False), wl.m - 1, 255, 256])
+    _check_fused(F, wl, (0, 1600), (1600, 4160), (4160, 8256), rows=rows)
+
+
 def test_fused_identity_range_bit_exact_when_accumulation_is_exact(F):
     rng = np.random.default_rng(22)
     M, N, K = 130, 256, 256

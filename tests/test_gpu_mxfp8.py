@@ -112,6 +112,18 @@ def test_gemm_ragged(F, m, n, k):
     _linear(F, synth.LinearWorkload(f"mx_{m}x{n}x{k}", m, k, n, seed=m + n + k))
 
 
+@pytest.mark.parametrize("m,n,k", [(2341, 2056, 3136), (4608, 3072, 1088)])
+def test_gemm_wide_tiles_ragged_sampled(F, m, n, k):
+    # shapes that take the 256 x 256 tiles: sampled rows and columns, the last
+    # ones and those at 128-row / 128-column boundaries included
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert ((m + 255) // 256) * ((n + 255) // 256) >= sms // 2
+    rng = np.random.default_rng(m + n)
+    rows = np.unique(np.r_[rng.choice(m, 40, replace=False), m - 1, 127, 128, 255, 256])
+    cols = np.unique(np.r_[rng.choice(n, 64, replace=False), n - 1, 127, 128, 255, 256])
+    _linear(F, synth.LinearWorkload(f"mx_wide_{m}x{n}x{k}", m, k, n, seed=m + n + k), rows=rows, cols=cols)
+
+
 def test_gemm_mlp_up_sampled(F):
     wl = synth.MLP_UP
     rng = np.random.default_rng(10)
