@@ -259,9 +259,11 @@ nvfp4_status nvfp4_mxfp8_quantize(const void* x, int64_t M, int64_t K, uint8_t* 
   nvfp4_status st = current_device(&dev);
   if (st != NVFP4_OK) return st;
   CUtensorMap tx;
-  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  const int tile_rows = quantize_tile_rows(M, K, dev->num_sms);
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, static_cast<uint32_t>(tile_rows),
+                 CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_quantize_mxfp8(tx, M, K, codes, sf, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_quantize_mxfp8(tx, tile_rows, M, K, codes, sf, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "mxfp8 quantize launch");
   return ok();
 }
@@ -365,9 +367,11 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
   nvfp4_status st = current_device(&dev);
   if (st != NVFP4_OK) return st;
   CUtensorMap tx;
-  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  const int tile_rows = quantize_tile_rows(M, K, dev->num_sms);
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, static_cast<uint32_t>(tile_rows),
+                 CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_quantize(tx, M, K, g, codes, sf, static_cast<cudaStream_t>(stream), *dev);
+  cudaError_t e = launch_quantize(tx, tile_rows, M, K, g, codes, sf, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return ok();
 }
@@ -388,9 +392,11 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t
   nvfp4_status st = current_device(&dev);
   if (st != NVFP4_OK) return st;
   CUtensorMap tx;
-  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  const int tile_rows = quantize_tile_rows(M, K, dev->num_sms);
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, static_cast<uint32_t>(tile_rows),
+                 CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
-  cudaError_t e = launch_quantize_dynamic(tx, x, M, K, codes, sf, scale_out, static_cast<uint32_t*>(workspace),
+  cudaError_t e = launch_quantize_dynamic(tx, tile_rows, x, M, K, codes, sf, scale_out, static_cast<uint32_t*>(workspace),
                                           static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
   return ok();
@@ -416,10 +422,12 @@ nvfp4_status nvfp4_quantize_dynamic_noalloc(const void* x, int64_t M, int64_t K,
   st = noalloc_scratch(dev->device, &scratch);
   if (st != NVFP4_OK) return st;
   CUtensorMap tx;
-  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  const int tile_rows = quantize_tile_rows(M, K, dev->num_sms);
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, static_cast<uint32_t>(tile_rows),
+                 CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
   // the launch zeroes the scratch on the stream before the kernel
-  cudaError_t e = launch_quantize_dynamic(tx, x, M, K, codes, sf, scale_out, scratch,
+  cudaError_t e = launch_quantize_dynamic(tx, tile_rows, x, M, K, codes, sf, scale_out, scratch,
                                           static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
   return ok();

@@ -59,16 +59,19 @@ struct DynamicScaleArgs {
 // Bytes of scratch one dynamic-scale quantize uses (zeroed by the launch).
 constexpr size_t kDynamicScratchBytes = 8;
 
-// tmap_x: bf16 [M, K], box 128 rows x 64 columns, 128-byte swizzle.
-cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
-                            cudaStream_t stream, const DeviceInfo& dev);
+// Rows of one quantize tile for a [M, K] input (128 or 256): the TMA box
+// height of the bf16 input's tensor map, passed back to the launch.
+int quantize_tile_rows(int64_t M, int64_t K, int num_sms);
+// tmap_x: bf16 [M, K], box tile_rows rows x 64 columns, 128-byte swizzle.
+cudaError_t launch_quantize(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, float g, uint8_t* codes,
+                            uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev);
 // MXFP8 (E4M3 codes [M, K], E8M0 scales, one per 32 elements, swizzled).
-cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
-                                  cudaStream_t stream, const DeviceInfo& dev);
+cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, uint8_t* codes,
+                                  uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev);
 // Same, with g measured on x in the same (cooperative) launch.
-cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, uint8_t* codes,
-                                    uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream,
-                                    const DeviceInfo& dev);
+cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, int tile_rows, const void* x, int64_t M, int64_t K,
+                                    uint8_t* codes, uint8_t* sf, float* scale_out, uint32_t* scratch,
+                                    cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_calibrate(const void* x, int64_t n, float* out, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out, cudaStream_t stream);
 

@@ -3,18 +3,19 @@
 // "Kernels": `nvfp4_quantize` runs on the activations at every forward).
 //
 // The quantize kernel is HBM-bound (2 bytes read, 0.5 + 1/16 bytes written per
-// element).  One persistent CTA per SM streams tiles of 128 rows x 64 columns
-// (16 KB of bf16, the width of one scale atom) through 12 TMA stages in
-// shared memory (192 KB in flight per SM), loaded with the 128-byte swizzle so
-// that 32 threads reading 32 different rows hit distinct banks.  Sixteen
-// consumer warps work independently, with no block-wide barrier: four groups
-// of four warps take every fourth tile, and warp q of a group owns rows
-// 32q..32q+31 of it.  Each group has its own three stages: an mbarrier wait
-// only tells phases apart by parity, so a stage must be consumed in order by
-// one consumer (a group running ahead on a shared ring could take a stage's
-// previous phase for its next one).  A thread owns one row's 64 elements (four 16-element
-// blocks), so it produces exactly one 4-byte word of the swizzled scale layout
-// and 32 bytes of codes.
+// element).  One persistent CTA per SM streams tiles of 256 rows x 64 columns
+// (32 KB of bf16, the width of one scale atom) through 6 TMA stages in shared
+// memory (192 KB in flight per SM), loaded with the 128-byte swizzle so that
+// 32 threads reading 32 different rows hit distinct banks.  24 consumer warps
+// work independently, with no block-wide barrier: three groups of eight warps
+// take every third tile, and warp q of a group owns rows 32q..32q+31 of it.
+// Each group has its own two stages: an mbarrier wait only tells phases apart
+// by parity, so a stage must be consumed in order by one consumer (a group
+// running ahead on a shared ring could take a stage's previous phase for its
+// next one).  A thread owns one row's 64 elements (four 16-element blocks),
+// so it produces exactly one 4-byte word of the swizzled scale layout and 32
+// bytes of codes, written as one whole 32-byte sector.  The consumers' work,
+// not HBM, set the pace with 16 warps; 24 keep more rows in flight.
 //
 // The dynamic variant measures the per-tensor scale in the same launch: every
 // CTA first takes max |x| over its own tiles (plain 16-byte loads), folds it
@@ -29,34 +30,45 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kQRows = 128;
-constexpr int kQCols = 64;
-constexpr int kQGroups = 4;                         // tiles processed concurrently per CTA
-constexpr int kQStagesPerGroup = 3;
-constexpr int kQStages = kQGroups * kQStagesPerGroup;
-constexpr int kQConsumerWarps = 4 * kQGroups;       // 4 quarter-warps per tile
-constexpr int kQThreads = (kQConsumerWarps + 1) * 32;  // + one producer warp
-constexpr uint32_t kQTileBytes = kQRows * kQCols * 2;  // 16 KB of bf16
-constexpr uint32_t kQOffBar = kQStages * kQTileBytes;
-constexpr uint32_t kQOffMax = kQOffBar + 2 * kQStages * 8 + 16;  // per-warp maxima of the amax pass
-constexpr uint32_t kQSmemBytes = kQOffMax + 32 * 4 + 1024;        // + alignment slack
+// Tile shape and ring of one launch: 128-row tiles (four groups of four
+// warps, three stages each) keep enough tiles per CTA in flight for small
+// tensors; 256-row tiles (three groups of eight warps, two stages each) put
+// 24 consumer warps to work on large ones.  Both hold 192 KB per SM.
+template <int kRows>
+struct QCfg {
+  static constexpr int kTileRows = kRows;
+  static constexpr int kCols = 64;
+  static constexpr int kGroups = kRows == 256 ? 3 : 4;       // tiles processed concurrently per CTA
+  static constexpr int kStagesPerGroup = kRows == 256 ? 2 : 3;
+  static constexpr int kStages = kGroups * kStagesPerGroup;
+  static constexpr int kWarpsPerTile = kRows / 32;           // one row per thread
+  static constexpr int kConsumerWarps = kWarpsPerTile * kGroups;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+  static constexpr uint32_t kTileBytes = kRows * kCols * 2;
+  static constexpr uint32_t kOffBar = kStages * kTileBytes;
+  static constexpr uint32_t kOffMax = kOffBar + 2 * kStages * 8 + 16;  // per-warp maxima of the amax pass
+  static constexpr uint32_t kSmemBytes = kOffMax + (kConsumerWarps + 1) * 4 + 1024;  // + alignment slack
+  static_assert(kRows == 128 || kRows == 256, "tile rows");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
-template <bool kDynamic, bool kMx>
-__global__ void __launch_bounds__(kQThreads, 1)
+template <bool kDynamic, bool kMx, int kRows>
+__global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
     quantize_kernel(const __grid_constant__ CUtensorMap tmap_x, int64_t M, int64_t K, float g,
                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int64_t tiles_k, int64_t n_tiles,
                     unsigned* fault_word, DynamicScaleArgs dyn) {
+  using Q = QCfg<kRows>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQOffBar);
-  uint64_t* empty = full + kQStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQStages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Q::kOffBar);
+  uint64_t* empty = full + Q::kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + Q::kStages);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
+    for (int s = 0; s < Q::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 4);  // the four quarter-warps of the tile
+      mbar_init(&empty[s], Q::kWarpsPerTile);  // every consumer warp of the tile
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -65,7 +77,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   unsigned fault = 0u;
   // This CTA's tiles are blockIdx.x + j * gridDim.x, j = 0 .. my_tiles-1.
   // The ring carries a sequence of n_seq loads, entry jj = 4i + g going to
-  // consumer group g, stage g * kQStagesPerGroup + i % 3.  The static variant
+  // consumer group g, stage g * Q::kStagesPerGroup + i % 3.  The static variant
   // loads each tile once (entry jj = tile j).  The dynamic one loads them
   // twice: entries 0 .. my_tiles-1 for the amax pass in order, then the
   // quantize pass in reverse order, so that its first tiles are the ones
@@ -77,43 +89,47 @@ __global__ void __launch_bounds__(kQThreads, 1)
     return blockIdx.x + j * gridDim.x;
   };
 
-  if (warp == kQConsumerWarps) {
+  if (warp == Q::kConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
       int64_t jj = 0;
       for (; jj < n_seq; ++jj) {
-        const int64_t i = jj / kQGroups;
-        const int stage = static_cast<int>(jj % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
-        const uint32_t phase = static_cast<uint32_t>((i / kQStagesPerGroup) & 1);
+        const int64_t i = jj / Q::kGroups;
+        const int stage = static_cast<int>(jj % Q::kGroups) * Q::kStagesPerGroup + static_cast<int>(i % Q::kStagesPerGroup);
+        const uint32_t phase = static_cast<uint32_t>((i / Q::kStagesPerGroup) & 1);
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
           fault = kFaultProducerWait;
           break;
         }
         const int64_t tile = seq_tile(jj);
-        mbar_arrive_expect_tx(&full[stage], kQTileBytes);
-        tma_load_2d(smem + stage * kQTileBytes, &tmap_x, &full[stage], static_cast<int32_t>((tile % tiles_k) * kQCols),
-                    static_cast<int32_t>((tile / tiles_k) * kQRows));
+        mbar_arrive_expect_tx(&full[stage], Q::kTileBytes);
+        tma_load_2d(smem + stage * Q::kTileBytes, &tmap_x, &full[stage], static_cast<int32_t>((tile % tiles_k) * Q::kCols),
+                    static_cast<int32_t>((tile / tiles_k) * Q::kTileRows));
       }
       if (fault != 0u) {
         *abort_flag = 1;
-        // let the copies already issued (the last kQStages entries) land
-        for (int64_t k = jj - 1; k >= 0 && k >= jj - kQStages; --k) {
-          const int64_t i = k / kQGroups;
-          const int stage = static_cast<int>(k % kQGroups) * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
-          mbar_wait(&full[stage], static_cast<uint32_t>((i / kQStagesPerGroup) & 1), nullptr);
+        // let the copies already issued (the last Q::kStages entries) land
+        for (int64_t k = jj - 1; k >= 0 && k >= jj - Q::kStages; --k) {
+          const int64_t i = k / Q::kGroups;
+          const int stage = static_cast<int>(k % Q::kGroups) * Q::kStagesPerGroup + static_cast<int>(i % Q::kStagesPerGroup);
+          mbar_wait(&full[stage], static_cast<uint32_t>((i / Q::kStagesPerGroup) & 1), nullptr);
         }
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const int group = warp >> 2;
-    const int q = warp & 3;         // rows 32q..32q+31 of each tile
-    const int rloc = q * 32 + lane; // this thread's row inside the tile
+    const int group = warp / Q::kWarpsPerTile;
+    const int q = warp % Q::kWarpsPerTile;  // rows 32q..32q+31 of each tile
+    const int rloc = q * 32 + lane;       // this thread's row inside the tile
+    const int64_t m_padded = (M + 127) & ~int64_t(127);  // rows of the scale buffer
     float amax_part = 0.0f;         // dynamic: max |x| over the rows this thread saw
     bool have_scale = !kDynamic;
     float d6 = __fmul_rn(6.0f, g);
     const int64_t katoms = K >> 6;
+    // 32-byte aligned codes rows (the usual case: every row starts at a
+    // multiple of 32 bytes when the buffer does) take one 32-byte store
+    const bool codes32 = (reinterpret_cast<uintptr_t>(codes) & 31u) == 0;
     const int64_t mx_katoms = (K / 32 + 3) / 4;  // MXFP8 scale atoms per 128-row block
 
     // Dynamic variant, once per consumer warp (every one of the 16 reaches
@@ -124,11 +140,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
       float m = amax_part;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      volatile float* warp_max = reinterpret_cast<volatile float*>(smem + kQOffMax);
+      volatile float* warp_max = reinterpret_cast<volatile float*>(smem + Q::kOffMax);
       if (lane == 0) warp_max[warp] = m;
-      named_barrier_sync(1, kQConsumerWarps * 32);
+      named_barrier_sync(1, Q::kConsumerWarps * 32);
       if (warp == 0 && lane == 0) {
-        for (int w = 1; w < kQConsumerWarps; ++w) m = fmaxf(m, warp_max[w]);
+        for (int w = 1; w < Q::kConsumerWarps; ++w) m = fmaxf(m, warp_max[w]);
         // |x| >= 0, so the float's bit pattern orders like the value
         atomicMax(dyn.scratch, __float_as_uint(m));
         __threadfence();
@@ -139,10 +155,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
           if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) break;
           __nanosleep(64);
         }
-        warp_max[kQConsumerWarps] = arrived >= gridDim.x ? __uint_as_float(ld_acquire_gpu(dyn.scratch)) : -1.0f;
+        warp_max[Q::kConsumerWarps] = arrived >= gridDim.x ? __uint_as_float(ld_acquire_gpu(dyn.scratch)) : -1.0f;
       }
-      named_barrier_sync(1, kQConsumerWarps * 32);
-      const float amax = warp_max[kQConsumerWarps];
+      named_barrier_sync(1, Q::kConsumerWarps * 32);
+      const float amax = warp_max[Q::kConsumerWarps];
       if (amax < 0.0f) {
         fault = kFaultGridWait;
         *abort_flag = 1;
@@ -158,21 +174,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
       return true;
     };
 
-    for (int64_t jj = group; jj < n_seq; jj += kQGroups) {
+    for (int64_t jj = group; jj < n_seq; jj += Q::kGroups) {
       if (!have_scale && jj >= my_tiles) {
         have_scale = true;
         if (!grid_scale()) break;
       }
-      const int64_t i = jj / kQGroups;
-      const int stage = group * kQStagesPerGroup + static_cast<int>(i % kQStagesPerGroup);
-      const uint32_t phase = static_cast<uint32_t>((i / kQStagesPerGroup) & 1);
+      const int64_t i = jj / Q::kGroups;
+      const int stage = group * Q::kStagesPerGroup + static_cast<int>(i % Q::kStagesPerGroup);
+      const uint32_t phase = static_cast<uint32_t>((i / Q::kStagesPerGroup) & 1);
       const bool got = mbar_wait(&full[stage], phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         fault = kFaultEpilogueWait;
         break;
       }
       // row rloc: 128 bytes, 16-byte chunk c stored at chunk c ^ (rloc % 8)
-      const uint8_t* row_s = smem + stage * kQTileBytes + rloc * 128;
+      const uint8_t* row_s = smem + stage * Q::kTileBytes + rloc * 128;
       uint4 v[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(row_s + ((c ^ (rloc & 7)) * 16));
@@ -196,7 +212,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       }
 
       const int64_t tile = seq_tile(jj);
-      const int64_t row = (tile / tiles_k) * kQRows + rloc;
+      const int64_t row = (tile / tiles_k) * Q::kTileRows + rloc;
       const int64_t katom = tile % tiles_k;  // 64-column group of the tile
       if constexpr (kMx) {
         // MXFP8: two 32-element blocks -> 64 E4M3 bytes and two E8M0 scale
@@ -225,17 +241,24 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
         if (row < M) {
           uint8_t* crow = codes + row * K + katom * 64;
+          if (codes32) {
+            st_global_v8(crow, *reinterpret_cast<const uint32_t(*)[8]>(cw));
+            st_global_v8(crow + 32, *reinterpret_cast<const uint32_t(*)[8]>(cw + 8));
+          } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(crow + 16 * c) = make_uint4(cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(crow + 16 * c) = make_uint4(cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
+          }
         }
         // rows past M: zero-filled data, amax 0, scale bytes 0 (the padding).
         // The last tile of a K that is 64 mod 128 also zeroes the two padding
         // columns of its word.
-        if ((katom & 1) == 0 && katom == tiles_k - 1)
-          *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 2, mx_katoms)) = sfh;
-        else
-          *reinterpret_cast<uint16_t*>(sf + sf_offset(row, katom * 2, mx_katoms)) = static_cast<uint16_t>(sfh);
+        if (row < m_padded) {
+          if ((katom & 1) == 0 && katom == tiles_k - 1)
+            *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 2, mx_katoms)) = sfh;
+          else
+            *reinterpret_cast<uint16_t*>(sf + sf_offset(row, katom * 2, mx_katoms)) = static_cast<uint16_t>(sfh);
+        }
         continue;
       }
       uint32_t sfw = 0u;
@@ -264,12 +287,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
       }
       if (row < M) {
         uint8_t* crow = codes + row * (K >> 1) + katom * 32;
-        *reinterpret_cast<uint4*>(crow) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        *reinterpret_cast<uint4*>(crow + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        if (codes32)  // one full 32-byte sector per thread
+          st_global_v8(crow, cw);
+        else {
+          *reinterpret_cast<uint4*>(crow) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint4*>(crow + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        }
       }
-      // rows past M belong to the zero padding of the scale buffer (their
-      // data was zero-filled by the TMA, so sfw == 0)
-      *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 4, katoms)) = sfw;
+      // rows past M up to the next multiple of 128 are the zero padding of
+      // the scale buffer (their data was zero-filled by the TMA, so sfw == 0)
+      if (row < m_padded) *reinterpret_cast<uint32_t*>(sf + sf_offset(row, katom * 4, katoms)) = sfw;
     }
     // a group whose entries ended inside the amax pass (or that gave up
     // there) still takes part in the CTA's scale exchange
@@ -306,51 +333,37 @@ __global__ void swizzle_sf_kernel(const uint8_t* __restrict__ sf_lin, int64_t ro
 
 }  // namespace
 
-cudaError_t launch_quantize(const CUtensorMap& tmap_x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
-                            cudaStream_t stream, const DeviceInfo& dev) {
-  const int64_t tiles_m = (M + kQRows - 1) / kQRows;
-  const int64_t tiles_k = (K + kQCols - 1) / kQCols;
-  const int64_t n_tiles = tiles_m * tiles_k;
-  const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
-  cudaError_t err =
-      cudaFuncSetAttribute(quantize_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
-  if (err != cudaSuccess) return err;
-  quantize_kernel<false, false><<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles,
-                                                                   dev.fault, DynamicScaleArgs{});
-  return cudaGetLastError();
+int quantize_tile_rows(int64_t M, int64_t K, int num_sms) {
+  // 256-row tiles once every CTA gets at least eight of them
+  const int64_t tiles256 = ((M + 255) / 256) * ((K + 63) / 64);
+  return tiles256 >= 8 * static_cast<int64_t>(num_sms) ? 256 : 128;
 }
 
-cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
-                                  cudaStream_t stream, const DeviceInfo& dev) {
-  const int64_t tiles_m = (M + kQRows - 1) / kQRows;
-  const int64_t tiles_k = (K + kQCols - 1) / kQCols;
-  const int64_t n_tiles = tiles_m * tiles_k;
-  const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
-  auto kernel = quantize_kernel<false, true>;
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
-  if (err != cudaSuccess) return err;
-  kernel<<<grid, kQThreads, kQSmemBytes, stream>>>(tmap_x, M, K, 0.0f, codes, sf, tiles_k, n_tiles, dev.fault,
-                                                   DynamicScaleArgs{});
-  return cudaGetLastError();
-}
+namespace {
 
-cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, uint8_t* codes,
-                                    uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream,
-                                    const DeviceInfo& dev) {
-  const int64_t tiles_m = (M + kQRows - 1) / kQRows;
-  const int64_t tiles_k = (K + kQCols - 1) / kQCols;
+template <bool kDynamic, bool kMx, int kRows>
+cudaError_t launch_q(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, float g, uint8_t* codes,
+                     uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream, const DeviceInfo& dev) {
+  using Q = QCfg<kRows>;
+  const int64_t tiles_m = (M + kRows - 1) / kRows;
+  const int64_t tiles_k = (K + Q::kCols - 1) / Q::kCols;
   const int64_t n_tiles = tiles_m * tiles_k;
   const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
-  auto kernel = quantize_kernel<true, false>;
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+  auto kernel = quantize_kernel<kDynamic, kMx, kRows>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::kSmemBytes);
   if (err != cudaSuccess) return err;
+  if (!kDynamic) {
+    kernel<<<grid, Q::kThreads, Q::kSmemBytes, stream>>>(tmap_x, M, K, g, codes, sf, tiles_k, n_tiles, dev.fault,
+                                                         DynamicScaleArgs{});
+    return cudaGetLastError();
+  }
   // the grid-wide maximum and the arrival counter start at zero
   err = cudaMemsetAsync(scratch, 0, kDynamicScratchBytes, stream);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kQThreads, 1, 1);
-  cfg.dynamicSmemBytes = kQSmemBytes;
+  cfg.blockDim = dim3(Q::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Q::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid-wide wait can complete
@@ -361,6 +374,28 @@ cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, const void* x, in
   err = cudaLaunchKernelEx(&cfg, kernel, tmap_x, M, K, 0.0f, codes, sf, tiles_k, n_tiles, dev.fault, dyn);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, float g, uint8_t* codes,
+                            uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev) {
+  return tile_rows == 256 ? launch_q<false, false, 256>(tmap_x, nullptr, M, K, g, codes, sf, nullptr, nullptr, stream, dev)
+                          : launch_q<false, false, 128>(tmap_x, nullptr, M, K, g, codes, sf, nullptr, nullptr, stream, dev);
+}
+
+cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, uint8_t* codes,
+                                  uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev) {
+  return tile_rows == 256 ? launch_q<false, true, 256>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, stream, dev)
+                          : launch_q<false, true, 128>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, stream, dev);
+}
+
+cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, int tile_rows, const void* x, int64_t M, int64_t K,
+                                    uint8_t* codes, uint8_t* sf, float* scale_out, uint32_t* scratch,
+                                    cudaStream_t stream, const DeviceInfo& dev) {
+  return tile_rows == 256
+             ? launch_q<true, false, 256>(tmap_x, x, M, K, 0.0f, codes, sf, scale_out, scratch, stream, dev)
+             : launch_q<true, false, 128>(tmap_x, x, M, K, 0.0f, codes, sf, scale_out, scratch, stream, dev);
 }
 
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out,

@@ -116,6 +116,42 @@ def test_special_blocks(F):
         _check_quant(F, xb, g, f"special g={g}")
 
 
+@pytest.mark.parametrize("m,k", [(4700, 12288), (4609, 15360), (4608, 12352)])
+def test_large_ragged_quantize_stays_inside_its_buffers(F, m, k):
+    # Shapes that take the 256-row tiles with M not a multiple of 256 (nor,
+    # for two of them, of 128): the last tile reaches past the scale buffer's
+    # padded rows, and must write neither codes nor scales there.  Both outputs
+    # sit inside larger buffers whose tails must stay untouched; sampled rows
+    # (the last ones included) are bit-exact and the padding rows are zero.
+    rng = np.random.default_rng(m + k)
+    x = synth.normal_bf16((m, k), 1.0, synth._gen(m + k))
+    g = float(O.global_scale(O.tensor_amax(f32(x))))
+    guard = 1 << 16
+    sf_bytes = F.nvfp4_sf_bytes(m, k)
+    codes_buf = torch.full((m * k // 2 + guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    sf_buf = torch.full((sf_bytes + guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    xd = x.cuda()
+    F.nvfp4_quantize(xd.data_ptr(), m, k, g, codes_buf.data_ptr(), sf_buf.data_ptr(),
+                     torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    F.nvfp4_check_fault()
+    assert torch.all(codes_buf[m * k // 2:] == 0xA5), "codes written past the buffer"
+    assert torch.all(sf_buf[sf_bytes:] == 0xA5), "scales written past the buffer"
+    rows = np.unique(np.r_[rng.choice(m, 48, replace=False), m - 1, m - 2, 4607, 4608])
+    rows = rows[rows < m]
+    xf = f32(x)[rows]
+    codes, sf = O.quantize_nvfp4(xf, np.float32(g))
+    got_codes = codes_buf[: m * k // 2].view(m, k // 2).cpu().numpy()[rows]
+    assert_bytes_equal(got_codes, codes, "codes")
+    sf_all = sf_buf[:sf_bytes].cpu().numpy()
+    r, c = np.meshgrid(rows, np.arange(k // 16), indexing="ij")
+    assert_bytes_equal(sf_all[O.sf_offset(r, c, k // 16)], sf, "scales")
+    mp = (m + 127) // 128 * 128
+    if mp > m:
+        r, c = np.meshgrid(np.arange(m, mp), np.arange(k // 16), indexing="ij")
+        assert np.all(sf_all[O.sf_offset(r, c, k // 16)] == 0), "scale padding rows"
+
+
 def test_quantize_is_deterministic(F):
     x = synth.laplace_activations(384, 3072, seed=77).cuda()
     a = F.quantize(x, 0.01)
