@@ -812,8 +812,14 @@ GemmConfig gemm_config(int64_t M, int64_t N, int num_sms) {
   // 256 x 256 tiles do a third more MMA work per pipeline step than 256 x 192
   // ones for the same per-k-tile synchronisation, but leave SMs idle when
   // there are fewer tiles than CTA pairs.
+  const int64_t pairs = num_sms / 2;
   const int64_t wide_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-  if (wide_tiles >= num_sms / 2) return GemmConfig{2, 256, 1};
+  if (wide_tiles >= pairs) return GemmConfig{2, 256, 1};
+  // Few tiles (a few hundred tokens): narrower 256 x 128 tiles put more CTA
+  // pairs to work as long as they still fit in one wave.
+  const int64_t tiles192 = ((M + 255) / 256) * ((N + 191) / 192);
+  const int64_t tiles128 = ((M + 255) / 256) * ((N + 127) / 128);
+  if (tiles192 < pairs && tiles128 <= pairs) return GemmConfig{2, 128, 2};
   return GemmConfig{2, 192, 2};
 }
 
@@ -825,6 +831,8 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
       return launch<2, 256, 1, false, true, true>(m, p, stream, dev);
     if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2)
       return launch<2, 192, 2, false, true, true>(m, p, stream, dev);
+    if (c.cta_group == 2 && c.tile_n == 128 && c.acc_bufs == 2)
+      return launch<2, 128, 2, false, true, true>(m, p, stream, dev);
     if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2)
       return launch<1, 192, 2, false, true, true>(m, p, stream, dev);
     return cudaErrorInvalidConfiguration;
@@ -833,6 +841,7 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
     if (fused) return cudaErrorInvalidConfiguration;
     if (c.cta_group == 2 && c.tile_n == 256 && c.acc_bufs == 1) return launch<2, 256, 1, false, true>(m, p, stream, dev);
     if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2) return launch<2, 192, 2, false, true>(m, p, stream, dev);
+    if (c.cta_group == 2 && c.tile_n == 128 && c.acc_bufs == 2) return launch<2, 128, 2, false, true>(m, p, stream, dev);
     if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2) return launch<1, 192, 2, false, true>(m, p, stream, dev);
     return cudaErrorInvalidConfiguration;
   }
@@ -842,6 +851,7 @@ cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const Gemm
                  : launch<CG, BN, ACC, false, false>(m, p, stream, dev);
   NVFP4_GEMM_CASE(2, 256, 1)
   NVFP4_GEMM_CASE(2, 192, 2)
+  NVFP4_GEMM_CASE(2, 128, 2)
   NVFP4_GEMM_CASE(1, 192, 2)
 #undef NVFP4_GEMM_CASE
   return cudaErrorInvalidConfiguration;

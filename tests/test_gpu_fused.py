@@ -119,6 +119,14 @@ def test_fused_single_stream_block_shape_sampled(F):
     _check_fused(F, wl, synth.SINGLE_Q, synth.SINGLE_KV, synth.SINGLE_MLP, rows=rows)
 
 
+def test_fused_256x192_tiles_sampled(F):
+    # about a thousand tokens: 256 x 192 tiles (too few for the wide ones, too
+    # many 256 x 128 ones for a single wave)
+    wl = synth.LinearWorkload("fused_mid", 1000, 1088, 2880, seed=24)
+    rows = np.unique(np.r_[np.random.default_rng(24).choice(wl.m, 40, replace=False), wl.m - 1, 255, 256])
+    _check_fused(F, wl, (0, 768), (768, 1408), (1408, 2880), rows=rows)
+
+
 def test_fused_wide_tiles_ragged_sampled(F):
     # A shape that takes the 256 x 256 tiles (at least one per CTA pair), ragged
     # in M and with range boundaries inside tiles and inside 128-column halves.

@@ -66,7 +66,7 @@ def test_tiny_workload(F):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 8, 64), (100, 200, 192), (129, 392, 320), (300, 64, 1024),
-                                   (128, 192, 256), (256, 384, 512), (77, 1000, 4096)])
+                                   (128, 192, 256), (256, 384, 512), (77, 1000, 4096), (1000, 3000, 1088)])
 def test_ragged_shapes(F, m, n, k):
     _check_linear(F, synth.LinearWorkload(f"ragged_{m}x{n}x{k}", m, k, n, seed=m + n + k))
 
