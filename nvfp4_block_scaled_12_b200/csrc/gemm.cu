@@ -599,11 +599,11 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
       tc_fence_after();
       const int row_base = (tm * kCG + static_cast<int>(rank)) * 128 + q * 32;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(h * 128);
+      // two 64-column loads: with four 32-column ones the compiler spilled
+      // parts of the slice to local memory (and the MLP-up GEMM ran 8% slower)
       uint32_t r[128];
-      tmem_ld_32x32b_x32(t_row + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
-      tmem_ld_32x32b_x32(t_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-      tmem_ld_32x32b_x32(t_row + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
-      tmem_ld_32x32b_x32(t_row + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+      tmem_ld_32x32b_x64(t_row, r);
+      tmem_ld_32x32b_x64(t_row + 64, r + 64);
       tmem_ld_wait_n<128>(r);
       // the accumulator is in registers: the next tile's MMAs may start
       tc_fence_before();
