@@ -118,7 +118,7 @@ struct Cfg {
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kFullTx = kCG * (kABytes + kBBytes);  // A/B bytes of the whole group
-  static_assert(kBN % 32 == 0 && kBN / kCG % 8 == 0, "tile width");
+  static_assert(kBN % 32 == 0 && kChunks * 32 == kBN && kBN / kCG % 8 == 0, "tile width");
   static_assert(kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
   static_assert(kSfSlots >= 2 && kSfSlots <= kStages, "TMEM budget");
   static_assert(kSfaCol % kSfaSlotCols == 0 && kSfbCol % 8 == 0 && kSfbSlotCols % 8 == 0, "tcgen05.st column alignment");
@@ -133,8 +133,6 @@ __device__ __forceinline__ float gelu_tanh_f32(float v) {
   return 0.5f * v * (1.0f + tanhf(u));
 }
 
-// Round to bf16 and back (the value the bf16 output holds).
-__device__ __forceinline__ float round_bf16(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
 // Stage 32 rows x 32 bf16 columns (this warp's slice of one chunk) in the
 // 64-byte-swizzled layout the Y tensor map expects, then TMA-store it.
