@@ -5,9 +5,7 @@
 // left unquantized).  Per element: v = fl(fl(e2m1(q) * e4m3(s)) * g) (the
 // first product is exact in fp32), then rounded to bf16.
 //
-// HBM-bound: 0.5 + 1/16 bytes in, 2 bytes out per element.  A thread turns
-// 4-byte code words (8 elements) into 16-byte bf16 chunks, so that a warp's
-// loads and stores are contiguous.
+// HBM-bound: 0.5 + 1/16 bytes in, 2 bytes out per element.
 #include <cuda_fp16.h>
 
 #include "internal.h"
@@ -35,34 +33,38 @@ __device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float (&f)[8]) {
   }
 }
 
-constexpr int kWordsPerThread = 4;
-
-__global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restrict__ codes,
+// One thread per 16 bytes of codes (32 elements, two 16-element blocks):
+// a 16-byte load, the blocks' two scale bytes as one 16-bit load (they are
+// adjacent bytes of the same swizzled scale word), and 64 bytes of bf16 out.
+// A warp reads 512 contiguous bytes of codes and writes 2 KB of output.
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint4* __restrict__ codes,
                                                          const uint8_t* __restrict__ sf, float g, int64_t K,
-                                                         int64_t row0, uint4* __restrict__ out) {
-  // grid: x = chunks of 256 * kWordsPerThread code words of a row, y = row - row0.
-  // Code word w of the row holds elements 8w .. 8w+7 and becomes 16 bytes of
-  // bf16; the threads of a warp take consecutive words, so its loads and
-  // stores are contiguous.
-  const int64_t row = row0 + blockIdx.y;
-  const int64_t words = K >> 3;
-  const int64_t katoms = K >> 6;
-  const uint32_t* cr = codes + row * words;
-  uint4* orow = out + row * words;
+                                                         int64_t n_chunks, bool out32, uint8_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n_chunks) return;
+  const int64_t per_row = K >> 5;
+  const int64_t row = i / per_row, c = i % per_row;
+  const uint4 w4 = codes[i];
+  const uint16_t sp = *reinterpret_cast<const uint16_t*>(sf + sf_offset(row, 2 * c, K >> 6));
+  const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
+  uint32_t packed[16];
 #pragma unroll
-  for (int u = 0; u < kWordsPerThread; ++u) {
-    const int64_t w_idx = (static_cast<int64_t>(blockIdx.x) * kWordsPerThread + u) * 256 + threadIdx.x;
-    if (w_idx < words) {
-      const uint32_t w = cr[w_idx];
-      const float s = e4m3_to_f32(sf[sf_offset(row, w_idx >> 1, katoms)]);
-      float f[8];
-      e2m1x8_to_f32(w, f);
-      uint32_t packed[4];
+  for (int u = 0; u < 4; ++u) {
+    const float s = e4m3_to_f32(u < 2 ? (sp & 0xFFu) : (sp >> 8));
+    float f[8];
+    e2m1x8_to_f32(words[u], f);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        packed[e] = pack_bf16x2(__fmul_rn(__fmul_rn(f[2 * e], s), g), __fmul_rn(__fmul_rn(f[2 * e + 1], s), g));
-      orow[w_idx] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    }
+    for (int e = 0; e < 4; ++e)
+      packed[4 * u + e] = pack_bf16x2(__fmul_rn(__fmul_rn(f[2 * e], s), g), __fmul_rn(__fmul_rn(f[2 * e + 1], s), g));
+  }
+  uint8_t* o = out + (row * K + 32 * c) * 2;
+  if (out32) {  // two whole 32-byte sectors
+    st_global_v8(o, *reinterpret_cast<const uint32_t(*)[8]>(packed));
+    st_global_v8(o + 32, *reinterpret_cast<const uint32_t(*)[8]>(packed + 8));
+  } else {
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      reinterpret_cast<uint4*>(o)[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
   }
 }
 
@@ -70,17 +72,13 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t* __restr
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* sf, float g, int64_t rows, int64_t K, void* out,
                               cudaStream_t stream) {
-  const int64_t words = K >> 3;
-  const int64_t per_block = 256 * kWordsPerThread;
-  for (int64_t r0 = 0; r0 < rows; r0 += 65535) {  // gridDim.y is at most 65535
-    const int64_t nr = rows - r0 < 65535 ? rows - r0 : 65535;
-    const dim3 grid(static_cast<unsigned>((words + per_block - 1) / per_block), static_cast<unsigned>(nr));
-    dequantize_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(codes), sf, g, K, r0,
-                                                  static_cast<uint4*>(out));
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  const int64_t n_chunks = rows * (K >> 5);
+  const int threads = 256;
+  const int64_t blocks = (n_chunks + threads - 1) / threads;
+  const bool out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  dequantize_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(codes), sf, g, K, n_chunks, out32, static_cast<uint8_t*>(out));
+  return cudaGetLastError();
 }
 
 }  // namespace nvfp4
