@@ -40,8 +40,11 @@ def test_tiny(F):
     _check_quant(F, synth.TINY.activations(), "tiny")
 
 
-@pytest.mark.parametrize("m,k", [(1, 64), (7, 192), (9, 320), (300, 4160), (33, 15360)])
+@pytest.mark.parametrize("m,k", [(1, 64), (7, 192), (9, 320), (300, 4160), (33, 15360),
+                                 (1, 1024), (9, 1024), (300, 2048), (17, 3072), (129, 4096), (5, 5120)])
 def test_ragged_shapes(F, m, k):
+    # K = 1024/2048/3072/4096 take the register-resident kernel, the rest the
+    # two-pass one
     _check_quant(F, synth.activations_with_outlier_channels(m, k, seed=m + k), f"ragged {m}x{k}")
 
 
@@ -54,6 +57,18 @@ def test_special_rows(F):
     x[4, 5] = 3.0                                  # a single non-zero element
     x[5, :] = 2.0 ** -130                          # bf16 subnormals
     _check_quant(F, torch.from_numpy(x).to(torch.bfloat16), "special")
+
+
+@pytest.mark.parametrize("k", [1024, 3072])
+def test_special_rows_register_path(F, k):
+    x = np.zeros((6, k), np.float32)
+    x[0, 7] = -0.0
+    x[1, :] = np.linspace(-1e30, 1e30, k)
+    x[2, :] = np.linspace(-1e-30, 1e-30, k)
+    x[3, :] = -np.logspace(-20, 20, k)
+    x[4, k - 1] = 3.0                              # the row's last element
+    x[5, :] = 2.0 ** -130
+    _check_quant(F, torch.from_numpy(x).to(torch.bfloat16), f"special K={k}")
 
 
 def test_mlp_up_activations_sampled_rows(F):
