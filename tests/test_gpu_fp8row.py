@@ -59,15 +59,23 @@ def test_special_rows(F):
     _check_quant(F, torch.from_numpy(x).to(torch.bfloat16), "special")
 
 
-@pytest.mark.parametrize("k", [1024, 3072])
+@pytest.mark.parametrize("k", [1024, 3072, 1088])
 def test_special_rows_register_path(F, k):
-    x = np.zeros((6, k), np.float32)
+    # row scales inside and outside the range of the kernels' branch-free
+    # division, signed zeros in zero and non-zero rows, quotients far below
+    # the smallest E4M3 subnormal
+    x = np.zeros((8, k), np.float32)
     x[0, 7] = -0.0
     x[1, :] = np.linspace(-1e30, 1e30, k)
     x[2, :] = np.linspace(-1e-30, 1e-30, k)
     x[3, :] = -np.logspace(-20, 20, k)
     x[4, k - 1] = 3.0                              # the row's last element
     x[5, :] = 2.0 ** -130
+    r = np.random.default_rng(k).laplace(size=k).astype(np.float32)
+    r[::7] = -0.0
+    r[3::11] = -(2.0 ** -133)
+    x[6, :] = r
+    x[7, :] = r * np.float32(2.0 ** 110)           # row scale above 2^100
     _check_quant(F, torch.from_numpy(x).to(torch.bfloat16), f"special K={k}")
 
 
