@@ -46,6 +46,10 @@
  *   - The current device must be compute capability 10.0 (B200, sm_100a);
  *     otherwise NVFP4_EARCH.  There is no CPU fallback.
  *   - K is a multiple of 64 and at least 64.
+ *   - Row counts (M, N, rows) and K are at most 2^30 - 1, which keeps every
+ *     row index and tile coordinate inside int32; larger sizes, and sizes
+ *     whose one-dimensional launch grid would exceed 2^31 - 1 blocks, return
+ *     NVFP4_EINVAL.
  *   - Per-tensor scales (g, alpha) must be finite; g must lie in
  *     [2^-64, 2^64] so that no intermediate of the quantizer overflows.
  */

@@ -152,11 +152,9 @@ nvfp4_status make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base,
   return make_tmap_nd(m, dt, base, 2, dims, strides, box, sw, what);
 }
 
-// Swizzled scale buffer of a [rows, k] tensor seen as [row blocks][k/64
-// atoms][128 x u32]; the box covers 4 atoms (one 256-wide k-tile) of
-// `box_blocks` row blocks.  Out-of-range atoms and blocks read as zero.
-// Swizzled scales as [row blocks][atoms][128 x u32]; one box = box_atoms
-// atoms of box_blocks row blocks.
+// Swizzled scale buffer of a [rows, k] tensor seen as [row blocks][atoms]
+// [128 x u32]; one box = box_atoms atoms (4 = one 256-wide NVFP4 k-tile) of
+// box_blocks row blocks.  Out-of-range atoms and blocks read as zero.
 nvfp4_status make_sf_tmap(CUtensorMap* m, const void* sf, int64_t rows, int64_t atoms, uint32_t box_atoms,
                           uint32_t box_blocks, const char* what) {
   const uint64_t dims[3] = {128, static_cast<uint64_t>(atoms), static_cast<uint64_t>((rows + 127) / 128)};
@@ -167,6 +165,24 @@ nvfp4_status make_sf_tmap(CUtensorMap* m, const void* sf, int64_t rows, int64_t 
 }
 
 bool finite_f(float v) { return isfinite(v) != 0; }
+
+// Largest row count and K of any entry point: keeps every row index and TMA
+// tile coordinate inside int32.
+constexpr int64_t kMaxDim = INT32_MAX / 2;
+
+// 1 <= rows <= kMaxDim; 64 <= K <= kMaxDim with K % 64 == 0.
+nvfp4_status check_rows_k(const char* rname, int64_t rows, const char* kname, int64_t K) {
+  if (rows < 1 || rows > kMaxDim)
+    return fail(NVFP4_EINVAL, "%s=%lld must be in [1, %lld]", rname, (long long)rows, (long long)kMaxDim);
+  if (K < 64 || K % 64 != 0 || K > kMaxDim)
+    return fail(NVFP4_EINVAL, "%s=%lld must be a positive multiple of 64, at most %lld", kname, (long long)K,
+                (long long)kMaxDim);
+  return NVFP4_OK;
+}
+
+// A one-dimensional grid of `threads`-thread blocks over `items` must fit
+// gridDim.x.
+bool grid_fits(int64_t items, int threads) { return (items + threads - 1) / threads <= INT32_MAX; }
 
 bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
 
@@ -179,15 +195,15 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          GemmConfig* cfg, const DeviceInfo** dev, bool mx = false, bool row = false,
                          bool fused = false) {
   if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
-  if (M < 1 || M > INT32_MAX / 2) return fail(NVFP4_EINVAL, "M=%lld out of range", (long long)M);
-  if (N < 8 || N % 8 != 0 || N > INT32_MAX / 2)
-    return fail(NVFP4_EINVAL, "N=%lld must be a positive multiple of 8", (long long)N);
-  if (K < 64 || K % 64 != 0 || K > INT32_MAX / 2)
-    return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  nvfp4_status st = check_rows_k("M", M, "K", K);
+  if (st != NVFP4_OK) return st;
+  if (N < 8 || N % 8 != 0 || N > kMaxDim)
+    return fail(NVFP4_EINVAL, "N=%lld must be a positive multiple of 8, at most %lld", (long long)N,
+                (long long)kMaxDim);
   if (!finite_f(alpha)) return fail(NVFP4_EINVAL, "alpha must be finite");
   if (!aligned16(a) || !aligned16(sfa) || !aligned16(b) || !aligned16(sfb) || !aligned16(bias))
     return fail(NVFP4_EALIGN, "operand pointers must be 16-byte aligned");
-  nvfp4_status st = current_device(dev);
+  st = current_device(dev);
   if (st != NVFP4_OK) return st;
 
   *cfg = gemm_config(M, N, (*dev)->num_sms);
@@ -251,8 +267,7 @@ size_t nvfp4_mxfp8_sf_bytes(int64_t rows, int64_t k) {
 
 nvfp4_status nvfp4_mxfp8_quantize(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf, void* stream) {
   if (!x || !codes || !sf) return fail(NVFP4_EINVAL, "null pointer");
-  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
-  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (check_rows_k("M", M, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
     return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
   const DeviceInfo* dev = nullptr;
@@ -288,8 +303,7 @@ nvfp4_status nvfp4_mxfp8_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_
 nvfp4_status nvfp4_fp8row_quantize(const void* x, int64_t M, int64_t K, uint8_t* codes, float* scale,
                                    void* stream) {
   if (!x || !codes || !scale) return fail(NVFP4_EINVAL, "null pointer");
-  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
-  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (check_rows_k("M", M, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scale))
     return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
   const DeviceInfo* dev = nullptr;
@@ -322,8 +336,8 @@ nvfp4_status nvfp4_fp8row_gemm(const uint8_t* a, const float* a_scale, const uin
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, float g, int64_t rows, int64_t K, void* out,
                               void* stream) {
   if (!codes || !sf || !out) return fail(NVFP4_EINVAL, "null pointer");
-  if (rows < 1) return fail(NVFP4_EINVAL, "rows=%lld must be >= 1", (long long)rows);
-  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (check_rows_k("rows", rows, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
+  if (!grid_fits(rows * (K / 32), 256)) return fail(NVFP4_EINVAL, "rows*K=%lld is too large", (long long)(rows * K));
   if (!finite_f(g)) return fail(NVFP4_EINVAL, "g must be finite");
   if (!aligned16(codes) || !aligned16(sf) || !aligned16(out))
     return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
@@ -358,8 +372,7 @@ nvfp4_status nvfp4_calibrate(const void* x, int64_t n, float* out, void* stream)
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* sf,
                             void* stream) {
   if (!x || !codes || !sf) return fail(NVFP4_EINVAL, "null pointer");
-  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
-  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (check_rows_k("M", M, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
   if (!scale_ok(g)) return fail(NVFP4_EINVAL, "g=%g must be finite and in [2^-64, 2^64]", (double)g);
   if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
     return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
@@ -379,8 +392,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
 nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
                                     float* scale_out, void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !codes || !sf || !scale_out || !workspace) return fail(NVFP4_EINVAL, "null pointer");
-  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
-  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (check_rows_k("M", M, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
   if (workspace_bytes < kDynamicScratchBytes)
     return fail(NVFP4_EINVAL, "workspace_bytes=%zu is below NVFP4_DYNAMIC_WORKSPACE_BYTES=%zu", workspace_bytes,
                 kDynamicScratchBytes);
@@ -405,8 +417,7 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t
 nvfp4_status nvfp4_quantize_dynamic_noalloc(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
                                             float* scale_out, void* stream) {
   if (!x || !codes || !sf || !scale_out) return fail(NVFP4_EINVAL, "null pointer");
-  if (M < 1) return fail(NVFP4_EINVAL, "M=%lld must be >= 1", (long long)M);
-  if (K < 64 || K % 64 != 0) return fail(NVFP4_EINVAL, "K=%lld must be a positive multiple of 64", (long long)K);
+  if (check_rows_k("M", M, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
     return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0) return fail(NVFP4_EALIGN, "scale_out must be 4-byte aligned");
@@ -436,8 +447,9 @@ nvfp4_status nvfp4_quantize_dynamic_noalloc(const void* x, int64_t M, int64_t K,
 nvfp4_status nvfp4_swizzle_sf(const uint8_t* sf_linear, int64_t rows, int64_t k, uint8_t* sf_swizzled,
                               void* stream) {
   if (!sf_linear || !sf_swizzled) return fail(NVFP4_EINVAL, "null pointer");
-  if (rows < 1) return fail(NVFP4_EINVAL, "rows=%lld must be >= 1", (long long)rows);
-  if (k < 64 || k % 64 != 0) return fail(NVFP4_EINVAL, "k=%lld must be a positive multiple of 64", (long long)k);
+  if (check_rows_k("rows", rows, "k", k) != NVFP4_OK) return NVFP4_EINVAL;
+  if (!grid_fits((rows + 127) / 128 * (k / 64) * 32, 256))
+    return fail(NVFP4_EINVAL, "rows*k=%lld is too large", (long long)(rows * k));
   if (!aligned16(sf_swizzled)) return fail(NVFP4_EALIGN, "sf_swizzled must be 16-byte aligned");
   const DeviceInfo* dev = nullptr;
   nvfp4_status st = current_device(&dev);

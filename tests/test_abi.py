@@ -139,6 +139,26 @@ def test_calibrate_and_swizzle_reject_bad_arguments_on_the_host():
     _expect(F.NVFP4_EALIGN, F.nvfp4_swizzle_sf, P, 4, 64, P + 4, 0)
 
 
+BIG = 1 << 30  # one past the largest row count or K
+
+
+def test_sizes_past_the_int32_limits_are_rejected_on_the_host():
+    W = F.NVFP4_DYNAMIC_WORKSPACE_BYTES
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, BIG, 64, 1.0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize, P, 4, BIG, 1.0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic, P, BIG, 64, P, P, P, P, W, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_dynamic_noalloc, P, 4, BIG, P, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_mxfp8_quantize, P, BIG, 64, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_fp8row_quantize, P, BIG, 64, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, BIG, 64, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, 16, BIG, 64, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm, P, P, P, P, 16, 64, BIG, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_dequantize, P, P, 1.0, BIG, 64, P, 0)
+    # rows and K each in range, but a grid of more than 2^31 - 1 blocks
+    _expect(F.NVFP4_EINVAL, F.nvfp4_dequantize, P, P, 1.0, BIG - 1, BIG - 64, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_swizzle_sf, P, BIG - 1, BIG - 64, P, 0)
+
+
 def test_valid_arguments_without_a_device_fail_loudly_not_silently():
     # On this CPU-only host a valid call reaches the device check and must
     # report an error: there is no CPU fallback.
