@@ -5,7 +5,9 @@ one (raw device pointers as ints, sizes, scales, a CUDA stream handle) and do
 argument marshalling only.  The helpers without the prefix (``quantize``,
 ``gemm``, ``gemm_quant``, ``swizzle_sf``) take torch tensors, allocate the
 outputs with torch (device memory is the only thing torch provides here) and
-call the same entry points on the current torch stream.  Every step of the
+call the same entry points on the current torch stream; every tensor they
+pass on, the caller's own output buffers included, is checked first (dtype,
+contiguity, current device, enough elements for what the kernel touches).  Every step of the
 computation runs in the library's CUDA kernels; there is no fallback: the
 first call raises ImportError if the library was not built.
 
@@ -194,7 +196,10 @@ def _ptr(t) -> int:
     return 0 if t is None else int(t.data_ptr())
 
 
-def _need(t, dtype, shape, name):
+def _need(t, dtype, shape, name, min_numel=None, dev=None):
+    """``t`` must be a contiguous CUDA tensor of ``dtype`` on the current
+    device, of ``shape`` (if given) and with at least ``min_numel`` elements
+    (if given): the library reads and writes through its raw pointer."""
     torch = _torch()
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
@@ -202,8 +207,27 @@ def _need(t, dtype, shape, name):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {min_numel} needed")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    dev = torch.cuda.current_device() if dev is None else dev
+    if t.device.index != dev:
+        raise ValueError(f"{name} is on {t.device}, the current device is cuda:{dev}")
+
+
+def _need_nvfp4(t, name, rows=None, k=None, dev=None):
+    """An NVFP4Tensor whose buffers hold ``rows`` x ``k`` elements (its own
+    rows and k when not given)."""
+    rows = t.rows if rows is None else rows
+    k = t.k if k is None else k
+    torch = _torch()
+    if (t.rows, t.k) != (rows, k):
+        raise ValueError(f"{name} is [{t.rows}, {t.k}], [{rows}, {k}] needed")
+    _need(t.codes, torch.uint8, None, f"{name}.codes", rows * k // 2, dev=dev)
+    _need(t.sf, torch.uint8, None, f"{name}.sf", nvfp4_sf_bytes(rows, k), dev=dev)
+    if t.g is None:  # the scale measured on the device: [amax, g]
+        _need(t.scale, torch.float32, None, f"{name}.scale", 2, dev=dev)
 
 
 @dataclass
@@ -224,7 +248,8 @@ def calibrate(x, stream=None):
     """Per-tensor scale of bf16 ``x`` on the GPU.  Returns a float32 CUDA
     tensor [amax, g] with g = amax / 2688 (nothing is read back)."""
     torch = _torch()
-    _need(x, torch.bfloat16, None, "x")
+    dev = torch.cuda.current_device()
+    _need(x, torch.bfloat16, None, "x", dev=dev)
     out = torch.empty(2, dtype=torch.float32, device=x.device)
     nvfp4_calibrate(_ptr(x), x.numel(), _ptr(out), _stream(stream))
     return out
@@ -238,11 +263,17 @@ def global_scale(x, stream=None) -> float:
 def quantize(x, g: float, out: Optional[NVFP4Tensor] = None, stream=None) -> NVFP4Tensor:
     """Quantize bf16 ``x`` [M, K] to NVFP4 with per-tensor decode scale g."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     M, K = x.shape
-    _need(x, torch.bfloat16, None, "x")
+    _need(x, torch.bfloat16, None, "x", dev=dev)
     if out is None:
         out = NVFP4Tensor(torch.empty(M, K // 2, dtype=torch.uint8, device=x.device),
                           torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=x.device), float(g), M, K)
+    else:
+        _need(out.codes, torch.uint8, None, "out.codes", M * K // 2, dev=dev)
+        _need(out.sf, torch.uint8, None, "out.sf", nvfp4_sf_bytes(M, K), dev=dev)
+        if (out.rows, out.k) != (M, K):
+            raise ValueError(f"out is [{out.rows}, {out.k}], x is [{M}, {K}]")
     nvfp4_quantize(_ptr(x), M, K, float(g), _ptr(out.codes), _ptr(out.sf), _stream(stream))
     out.g = float(g)
     return out
@@ -253,15 +284,23 @@ def quantize_dynamic(x, out: Optional[NVFP4Tensor] = None, workspace=None, strea
     the same launch (g = amax/2688, clamped; nothing is read back).  The
     result's ``scale`` holds [amax, g] on the device."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     M, K = x.shape
-    _need(x, torch.bfloat16, None, "x")
+    _need(x, torch.bfloat16, None, "x", dev=dev)
     if out is None:
         out = NVFP4Tensor(torch.empty(M, K // 2, dtype=torch.uint8, device=x.device),
                           torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=x.device), None, M, K)
+    else:
+        _need(out.codes, torch.uint8, None, "out.codes", M * K // 2, dev=dev)
+        _need(out.sf, torch.uint8, None, "out.sf", nvfp4_sf_bytes(M, K), dev=dev)
+        if (out.rows, out.k) != (M, K):
+            raise ValueError(f"out is [{out.rows}, {out.k}], x is [{M}, {K}]")
     if out.scale is None:
         out.scale = torch.empty(2, dtype=torch.float32, device=x.device)
+    _need(out.scale, torch.float32, None, "out.scale", 2, dev=dev)
     if workspace is None:
         workspace = torch.empty(NVFP4_DYNAMIC_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
+    _need(workspace, workspace.dtype, None, "workspace", dev=dev)
     nvfp4_quantize_dynamic(_ptr(x), M, K, _ptr(out.codes), _ptr(out.sf), _ptr(out.scale), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream))
     out.g = None
@@ -278,14 +317,27 @@ class MXFP8Tensor:
     k: int
 
 
+def _need_mxfp8(t, name, rows=None, k=None, dev=None):
+    rows = t.rows if rows is None else rows
+    k = t.k if k is None else k
+    torch = _torch()
+    if (t.rows, t.k) != (rows, k):
+        raise ValueError(f"{name} is [{t.rows}, {t.k}], [{rows}, {k}] needed")
+    _need(t.codes, torch.uint8, None, f"{name}.codes", rows * k, dev=dev)
+    _need(t.sf, torch.uint8, None, f"{name}.sf", nvfp4_mxfp8_sf_bytes(rows, k), dev=dev)
+
+
 def quantize_mxfp8(x, out: Optional[MXFP8Tensor] = None, stream=None) -> MXFP8Tensor:
     """Quantize bf16 ``x`` [M, K] to MXFP8 (power-of-two block scales)."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     M, K = x.shape
-    _need(x, torch.bfloat16, None, "x")
+    _need(x, torch.bfloat16, None, "x", dev=dev)
     if out is None:
         out = MXFP8Tensor(torch.empty(M, K, dtype=torch.uint8, device=x.device),
                           torch.empty(nvfp4_mxfp8_sf_bytes(M, K), dtype=torch.uint8, device=x.device), M, K)
+    else:
+        _need_mxfp8(out, "out", M, K, dev=dev)
     nvfp4_mxfp8_quantize(_ptr(x), M, K, _ptr(out.codes), _ptr(out.sf), _stream(stream))
     return out
 
@@ -293,13 +345,17 @@ def quantize_mxfp8(x, out: Optional[MXFP8Tensor] = None, stream=None) -> MXFP8Te
 def gemm_mxfp8(a: MXFP8Tensor, b: MXFP8Tensor, bias=None, alpha: float = 1.0, y=None, stream=None):
     """y = bf16(alpha * a_hat @ b_hat^T + bias) for MXFP8 operands."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     if a.k != b.k:
         raise ValueError("K mismatch")
     M, N, K = a.rows, b.rows, a.k
+    _need_mxfp8(a, "a", dev=dev)
+    _need_mxfp8(b, "b", dev=dev)
     if bias is not None:
-        _need(bias, torch.bfloat16, (N,), "bias")
+        _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _need(y, torch.bfloat16, (M, N), "y", dev=dev)
     nvfp4_mxfp8_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias),
                      _ptr(y), _stream(stream))
     return y
@@ -315,14 +371,27 @@ class FP8RowTensor:
     k: int
 
 
+def _need_fp8row(t, name, rows=None, k=None, dev=None):
+    rows = t.rows if rows is None else rows
+    k = t.k if k is None else k
+    torch = _torch()
+    if (t.rows, t.k) != (rows, k):
+        raise ValueError(f"{name} is [{t.rows}, {t.k}], [{rows}, {k}] needed")
+    _need(t.codes, torch.uint8, None, f"{name}.codes", rows * k, dev=dev)
+    _need(t.scale, torch.float32, None, f"{name}.scale", rows, dev=dev)
+
+
 def quantize_fp8row(x, out: Optional[FP8RowTensor] = None, stream=None) -> FP8RowTensor:
     """Quantize bf16 ``x`` [M, K] to E4M3 with one absmax scale per row."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     M, K = x.shape
-    _need(x, torch.bfloat16, None, "x")
+    _need(x, torch.bfloat16, None, "x", dev=dev)
     if out is None:
         out = FP8RowTensor(torch.empty(M, K, dtype=torch.uint8, device=x.device),
                            torch.empty(M, dtype=torch.float32, device=x.device), M, K)
+    else:
+        _need_fp8row(out, "out", M, K, dev=dev)
     nvfp4_fp8row_quantize(_ptr(x), M, K, _ptr(out.codes), _ptr(out.scale), _stream(stream))
     return out
 
@@ -330,13 +399,17 @@ def quantize_fp8row(x, out: Optional[FP8RowTensor] = None, stream=None) -> FP8Ro
 def gemm_fp8row(a: FP8RowTensor, b: FP8RowTensor, bias=None, y=None, stream=None):
     """y = bf16(a_scale[m] * b_scale[n] * a_q @ b_q^T + bias)."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     if a.k != b.k:
         raise ValueError("K mismatch")
     M, N, K = a.rows, b.rows, a.k
+    _need_fp8row(a, "a", dev=dev)
+    _need_fp8row(b, "b", dev=dev)
     if bias is not None:
-        _need(bias, torch.bfloat16, (N,), "bias")
+        _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _need(y, torch.bfloat16, (M, N), "y", dev=dev)
     nvfp4_fp8row_gemm(_ptr(a.codes), _ptr(a.scale), _ptr(b.codes), _ptr(b.scale), M, N, K, _ptr(bias), _ptr(y),
                       _stream(stream))
     return y
@@ -345,8 +418,13 @@ def gemm_fp8row(a: FP8RowTensor, b: FP8RowTensor, bias=None, y=None, stream=None
 def dequantize(t: NVFP4Tensor, out=None, stream=None):
     """NVFP4 tensor -> bf16 [rows, k] (the W4A16 path's weight)."""
     torch = _torch()
+    dev = torch.cuda.current_device()
+    if t.g is None:
+        raise ValueError("dequantize needs the per-tensor scale g on the host")
+    _need_nvfp4(t, "t", dev=dev)
     if out is None:
         out = torch.empty(t.rows, t.k, dtype=torch.bfloat16, device=t.codes.device)
+    _need(out, torch.bfloat16, (t.rows, t.k), "out", dev=dev)
     nvfp4_dequantize(_ptr(t.codes), _ptr(t.sf), float(t.g), t.rows, t.k, _ptr(out), _stream(stream))
     return out
 
@@ -363,7 +441,8 @@ def linear_w4a16(x, w: NVFP4Tensor, bias=None, w_bf16=None, stream=None):
 def swizzle_sf(sf_linear, rows: int, k: int, stream=None):
     """ModelOpt row-major E4M3 scales [rows, k/16] -> swizzled buffer."""
     torch = _torch()
-    _need(sf_linear, torch.uint8, (rows, k // 16), "sf_linear")
+    dev = torch.cuda.current_device()
+    _need(sf_linear, torch.uint8, (rows, k // 16), "sf_linear", dev=dev)
     out = torch.empty(nvfp4_sf_bytes(rows, k), dtype=torch.uint8, device=sf_linear.device)
     nvfp4_swizzle_sf(_ptr(sf_linear), rows, k, _ptr(out), _stream(stream))
     return out
@@ -372,16 +451,22 @@ def swizzle_sf(sf_linear, rows: int, k: int, stream=None):
 def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = None, y=None, stream=None):
     """y = bf16(alpha * a_hat @ b_hat^T + bias); alpha defaults to fl32(a.g * b.g)."""
     torch = _torch()
+    dev = torch.cuda.current_device()
     import numpy as np
     if a.k != b.k:
         raise ValueError("K mismatch")
     M, N, K = a.rows, b.rows, a.k
+    if alpha is None and b.g is None:
+        raise ValueError("the weight b needs its per-tensor scale g on the host, or pass alpha")
+    _need_nvfp4(a, "a", dev=dev)
+    _need_nvfp4(b, "b", dev=dev)
     if alpha is None and a.g is not None:
         alpha = float(np.float32(a.g) * np.float32(b.g))
     if bias is not None:
-        _need(bias, torch.bfloat16, (N,), "bias")
+        _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
+    _need(y, torch.bfloat16, (M, N), "y", dev=dev)
     if a.g is None and alpha is None:
         # the activation's scale lives on the device: alpha = fl32(g_a * g_b) in the kernel
         nvfp4_gemm_dynamic(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(b.g),
@@ -398,9 +483,28 @@ def gemm_quant(a: NVFP4Tensor, b: NVFP4Tensor, ranges: Sequence[tuple], *, bias=
     quantizes them into the next layer's NVFP4 input.  ``ranges`` holds
     ``(begin, end, act, dst, dst_col)`` tuples."""
     import numpy as np
+    torch = _torch()
+    dev = torch.cuda.current_device()
+    if a.k != b.k:
+        raise ValueError("K mismatch")
     M, N, K = a.rows, b.rows, a.k
+    _need_nvfp4(a, "a", dev=dev)
+    _need_nvfp4(b, "b", dev=dev)
     if alpha is None:
+        if a.g is None or b.g is None:
+            raise ValueError("gemm_quant needs alpha, or both per-tensor scales on the host")
         alpha = float(np.float32(a.g) * np.float32(b.g))
+    if bias is not None:
+        _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
+    if y_bf16 is not None:
+        _need(y_bf16, torch.bfloat16, None, "y_bf16", dev=dev)
+        if y_bf16.dim() != 2 or y_bf16.shape[0] < M:
+            raise ValueError(f"y_bf16 must be 2-D with at least {M} rows, got {tuple(y_bf16.shape)}")
+    if next_out is not None:
+        _need(next_out.codes, torch.uint8, None, "next_out.codes", M * next_out.k // 2, dev=dev)
+        _need(next_out.sf, torch.uint8, None, "next_out.sf", nvfp4_sf_bytes(M, next_out.k), dev=dev)
+        if next_out.rows != M:
+            raise ValueError(f"next_out has {next_out.rows} rows, the GEMM writes {M}")
     rs = [ColRange(int(r[0]), int(r[1]), int(r[2]), int(r[3]), int(r[4])) for r in ranges]
     ldy = int(y_bf16.shape[1]) if y_bf16 is not None else 0
     codes_next = next_out.codes if next_out is not None else None
