@@ -366,6 +366,30 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, float g,
  */
 nvfp4_status nvfp4_check_fault(void);
 
+/*
+ * Launch shapes the library picks, for callers that size work around them
+ * and for tests (host only: nothing touches a device).  Every GEMM entry point
+ * (NVFP4, fused, dynamic, MXFP8, row-wise FP8) takes the same tile shape for
+ * the same M, N and SM count:
+ *   out[0] = CTAs per output tile (1, or 2 for a CTA pair),
+ *   out[1] = tile width in output columns (128, 192 or 256),
+ *   out[2] = accumulator buffers in TMEM (1 or 2);
+ * the tile height is 128 * out[0] rows.  The rule: M <= 128 takes one CTA and
+ * 192 columns; otherwise 256 x 256 pair tiles when there are at least
+ * num_sms / 2 of them, else 256 x 128 when those still fit in one wave and
+ * 256 x 192 ones would not fill it, else 256 x 192.
+ * Errors: EINVAL (null out, M or N out of range, num_sms < 2).
+ */
+nvfp4_status nvfp4_gemm_tile_shape(int64_t M, int64_t N, int32_t num_sms, int32_t* out);
+
+/*
+ * Rows per tile of the NVFP4 and MXFP8 quantizers for an [M, K] input on a
+ * device with num_sms SMs: 256 once every SM gets at least eight 256-row
+ * tiles of 64 columns, else 128.  0 for invalid sizes (M or K out of range,
+ * K not a multiple of 64, num_sms < 1).  Host only.
+ */
+int32_t nvfp4_quantize_tile_rows(int64_t M, int64_t K, int32_t num_sms);
+
 /* Message describing the last error of the calling thread ("" if none).
  * The pointer stays valid until the thread's next call into the library. */
 const char* nvfp4_last_error(void);

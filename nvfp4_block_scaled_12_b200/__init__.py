@@ -70,10 +70,13 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_fp8row_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
     lib.nvfp4_dequantize.argtypes = [vp, vp, f32, i64, i64, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
+    lib.nvfp4_gemm_tile_shape.argtypes = [i64, i64, i32, ctypes.POINTER(ctypes.c_int32)]
+    lib.nvfp4_quantize_tile_rows.argtypes = [i64, i64, i32]
+    lib.nvfp4_quantize_tile_rows.restype = ctypes.c_int32
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
                  "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
-                 "nvfp4_dequantize", "nvfp4_check_fault"):
+                 "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_gemm_tile_shape"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -171,6 +174,17 @@ def nvfp4_dequantize(codes: int, sf: int, g: float, rows: int, K: int, out: int,
 
 def nvfp4_check_fault() -> None:
     _check(library().nvfp4_check_fault())
+
+
+def nvfp4_gemm_tile_shape(M: int, N: int, num_sms: int) -> tuple:
+    """(CTAs per tile, tile width, accumulator buffers) the GEMMs take for M x N."""
+    out = (ctypes.c_int32 * 3)()
+    _check(library().nvfp4_gemm_tile_shape(M, N, num_sms, out))
+    return tuple(out)
+
+
+def nvfp4_quantize_tile_rows(M: int, K: int, num_sms: int) -> int:
+    return int(library().nvfp4_quantize_tile_rows(M, K, num_sms))
 
 
 def nvfp4_last_error() -> str:

@@ -587,6 +587,22 @@ nvfp4_status nvfp4_check_fault(void) {
   return ok();
 }
 
+nvfp4_status nvfp4_gemm_tile_shape(int64_t M, int64_t N, int32_t num_sms, int32_t* out) {
+  if (!out) return fail(NVFP4_EINVAL, "null output pointer");
+  if (M < 1 || M > kMaxDim || N < 8 || N > kMaxDim || num_sms < 2)
+    return fail(NVFP4_EINVAL, "M=%lld, N=%lld, num_sms=%d out of range", (long long)M, (long long)N, num_sms);
+  const GemmConfig c = gemm_config(M, N, num_sms);
+  out[0] = c.cta_group;
+  out[1] = c.tile_n;
+  out[2] = c.acc_bufs;
+  return ok();
+}
+
+int32_t nvfp4_quantize_tile_rows(int64_t M, int64_t K, int32_t num_sms) {
+  if (M < 1 || M > kMaxDim || K < 64 || K % 64 != 0 || K > kMaxDim || num_sms < 1) return 0;
+  return quantize_tile_rows(M, K, num_sms);
+}
+
 const char* nvfp4_last_error(void) { return t_last_error.c_str(); }
 
 }  // extern "C"

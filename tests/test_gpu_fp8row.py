@@ -114,7 +114,7 @@ def test_gemm_wide_tiles_ragged_sampled(F, m, n, k):
     # shapes that take the 256 x 256 tiles: sampled rows and columns, the last
     # ones and those at 128-row / 128-column boundaries included
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert ((m + 255) // 256) * ((n + 255) // 256) >= sms // 2
+    assert F.nvfp4_gemm_tile_shape(m, n, sms) == (2, 256, 1)
     rng = np.random.default_rng(m + n)
     rows = np.unique(np.r_[rng.choice(m, 40, replace=False), m - 1, 127, 128, 255, 256])
     cols = np.unique(np.r_[rng.choice(n, 64, replace=False), n - 1, 127, 128, 255, 256])

@@ -123,6 +123,8 @@ def test_fused_256x192_tiles_sampled(F):
     # about a thousand tokens: 256 x 192 tiles (too few for the wide ones, too
     # many 256 x 128 ones for a single wave)
     wl = synth.LinearWorkload("fused_mid", 1000, 1088, 2880, seed=24)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert F.nvfp4_gemm_tile_shape(wl.m, wl.n, sms) == (2, 192, 2)
     rows = np.unique(np.r_[np.random.default_rng(24).choice(wl.m, 40, replace=False), wl.m - 1, 255, 256])
     _check_fused(F, wl, (0, 768), (768, 1408), (1408, 2880), rows=rows)
 
@@ -132,7 +134,7 @@ def test_fused_wide_tiles_ragged_sampled(F):
     # in M and with range boundaries inside tiles and inside 128-column halves.
     wl = synth.LinearWorkload("fused_wide", 2341, 1088, 8288, seed=23)  # columns 8256.. in no range
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert ((wl.m + 255) // 256) * ((wl.n + 255) // 256) >= sms // 2
+    assert F.nvfp4_gemm_tile_shape(wl.m, wl.n, sms) == (2, 256, 1)
     rows = np.unique(np.r_[np.random.default_rng(23).choice(wl.m, 40, replace=False), wl.m - 1, 255, 256])
     _check_fused(F, wl, (0, 1600), (1600, 4160), (4160, 8256), rows=rows)
 

@@ -162,9 +162,10 @@ def test_gemm_is_deterministic(F):
 
 def _wide(M, N):
     """True when the library takes its 256 x 256 CTA-pair tiles for this
-    plain NVFP4 GEMM: at least one tile per CTA pair of the device."""
+    GEMM on this device."""
+    import nvfp4_block_scaled_12_b200 as F
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    return ((M + 255) // 256) * ((N + 255) // 256) >= sms // 2
+    return F.nvfp4_gemm_tile_shape(M, N, sms) == (2, 256, 1)
 
 
 @pytest.mark.parametrize("m,n,k", [(2341, 2056, 3136), (4608, 3072, 3072), (2305, 8200, 1088)])

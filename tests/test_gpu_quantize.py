@@ -123,6 +123,8 @@ def test_large_ragged_quantize_stays_inside_its_buffers(F, m, k):
     # padded rows, and must write neither codes nor scales there.  Both outputs
     # sit inside larger buffers whose tails must stay untouched; sampled rows
     # (the last ones included) are bit-exact and the padding rows are zero.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert F.nvfp4_quantize_tile_rows(m, k, sms) == 256
     rng = np.random.default_rng(m + k)
     x = synth.normal_bf16((m, k), 1.0, synth._gen(m + k))
     g = float(O.global_scale(O.tensor_amax(f32(x))))
