@@ -290,18 +290,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
-// Bring [src, src + bytes) into L2 (no shared-memory destination); bytes is
-// a multiple of 16 and src 16-byte aligned.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
                ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(x), "r"(y)
@@ -387,12 +375,6 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask)
       : "memory");
 }
 
-// Copy a 32-row x 128-bit block from shared memory into TMEM lanes 0-31 at
-// column taddr..taddr+3, replicated into all four 32-lane sub-partitions.
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 // D (TMEM, fp32) (+)= A * B with NVFP4 operands: E2M1 elements from shared
 // memory and one UE4M3 scale per 16 elements from TMEM.  M=128, K=64.
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -425,15 +407,6 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(1024 >> 4) << 32;  // stride byte offset: 8 rows x 128 B
   d |= static_cast<uint64_t>(1) << 46;          // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;          // layout: 128-byte swizzle
-  return d;
-}
-
-// Descriptor of a plain (unswizzled) 32-row x 16-byte block, rows contiguous:
-// the source of tc_cp_32x128b_warpx4 for one 512-byte scale-factor atom.
-__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
-  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>(128 >> 4) << 32;  // stride byte offset: 8 rows x 16 B
-  d |= static_cast<uint64_t>(1) << 46;
   return d;
 }
 

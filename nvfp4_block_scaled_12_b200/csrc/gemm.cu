@@ -4,14 +4,16 @@
 // epilogue and an optional fused epilogue that quantizes the result for the
 // next layer.
 //
-// One persistent kernel, templated on the tile shape:
+// One persistent kernel, templated on the tile shape (the same rule for the
+// NVFP4, fused, MXFP8 and row-wise FP8 GEMMs; gemm_config below):
 //   256 x 256 (wide)  a CTA pair (cluster of 2) owns the tile: each CTA loads
 //            its 128 rows of A and 128 rows of B, and the pair leader issues
 //            tcgen05.mma.cta_group::2 (M=256, N=256, K=64) into one
-//            256-column accumulator.  Used for plain NVFP4 GEMMs with at
-//            least one tile per CTA pair.
+//            256-column accumulator.  Used with at least one tile per pair.
 //   256 x 192  a CTA pair with 96 rows of B per CTA and two accumulators
-//            (M > 128 otherwise, MXFP8, row-wise FP8, the fused epilogue).
+//            (M > 128 with fewer wide tiles than pairs).
+//   256 x 128  as 256 x 192 with 64 rows of B per CTA, when these tiles still
+//            fit in one wave and the 192-wide ones would leave pairs idle.
 //   128 x 192  one CTA per tile (M <= 128).
 // Every pipeline step (one 128-byte k-tile: four MMAs) costs the MMA-issuing
 // thread a barrier wait, a commit and its bookkeeping, during which the
