@@ -72,6 +72,32 @@ def gemm_dram_traffic():
         return None
 
 
+QUANT_PROFILE = os.path.join(PROFILES, "quantize_laplace_m4608_k12288.txt")
+QUANT_SOURCES = ("quantize.cu", "device.cuh", "internal.h")
+
+
+def quantize_dram_traffic():
+    """DRAM bytes per launch of the standalone quantize from the committed
+    ncu summary, or None when the kernel's sources changed since."""
+    try:
+        import hashlib
+        fields = {}
+        with open(QUANT_PROFILE) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        h = hashlib.sha256()
+        for name in QUANT_SOURCES:
+            with open(os.path.join(ROOT, "nvfp4_block_scaled_12_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if fields.get("sources_sha256") != h.hexdigest():
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -232,6 +258,35 @@ def cpu_baseline(budget_s: float = 10.0, rows: int = 256):
                       f"M=4608,K=3072,N=12288 (quantize + fp64 GEMM + bias), {total_t:.1f} s"}
 
 
+def quantize_cpu_baseline(budget_s: float = 8.0):
+    """The oracle's quantizer as it stands (numpy, elementwise: one core) on
+    the whole standalone-quantize workload bf16 [4608, 12288], swizzled scales
+    included, repeated until about ``budget_s`` seconds; GB/s on the same
+    2.5625 bytes per element as the GPU figure."""
+    import oracle as O
+    import synth
+    x = synth_cache("xq", lambda: synth.quantize_input().float().numpy())
+    g = O.global_scale(O.tensor_amax(x))
+    total, n = 0.0, 0
+    while total < budget_s and n < 8:
+        t0 = time.perf_counter()
+        _, sf = O.quantize_nvfp4(x, g)
+        O.swizzle_sf(sf)
+        total += time.perf_counter() - t0
+        n += 1
+    gbs = n * x.size * QUANT_BYTES_PER_ELEM / total / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} full passes over bf16 [4608,12288] (codes + swizzled scales), {total:.1f} s; "
+                      "numpy elementwise, one core"}
+
+
+def single_stream_g_next() -> float:
+    """The output projection's calibrated input scale of the single-stream
+    pair, stored by tests/golden/make_golden.py (computed by the oracle)."""
+    with open(os.path.join(ROOT, "tests", "golden", "single_stream_pair.json")) as f:
+        return float(json.load(f)["g_next"])
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -285,7 +340,8 @@ def extra_workloads(F, torch, synth, device, stream, median_ms, hbm, fp4_peak):
     w2q = F.quantize(w2, F.global_scale(w2))
     del w1, w2
     k2 = w2l.k
-    g2 = 0.05  # the output projection's static input scale
+    g2 = single_stream_g_next()  # the output projection's calibrated input scale
+    b2 = w2l.bias_vec().to(device)
     a2 = F.NVFP4Tensor(torch.empty(M, k2 // 2, dtype=torch.uint8, device=device),
                        torch.empty(F.nvfp4_sf_bytes(M, k2), dtype=torch.uint8, device=device), g2, M, k2)
     y_kv = torch.empty(M, kv1 - kv0, dtype=torch.bfloat16, device=device)
@@ -304,7 +360,7 @@ def extra_workloads(F, torch, synth, device, stream, median_ms, hbm, fp4_peak):
         F.gemm_quant(xq, w1q, bf16_ranges, y_bf16=y_all, stream=stream)
 
     def gemm2():
-        F.gemm(a2, w2q, y=y2, stream=stream)
+        F.gemm(a2, w2q, bias=b2, y=y2, stream=stream)
 
     def unfused():
         gemm1_bf16()
@@ -322,8 +378,9 @@ def extra_workloads(F, torch, synth, device, stream, median_ms, hbm, fp4_peak):
         "gemm1_fused_ms": t1f, "gemm1_fused_tflops": f1 / (t1f * 1e-3) / 1e12,
         "gemm1_bf16_out_ms": t1b, "gemm2_ms": t2, "gemm2_tflops": f2 / (t2 * 1e-3) / 1e12,
         "pair_fused_ms": tf, "pair_unfused_ms": tu,
-        "note": "GEMM1 4608x3072x21504 (Q, GELU(MLP) -> NVFP4 in the epilogue; K,V -> bf16), GEMM2 "
-                "4608x15360x3072; unfused = GEMM1 writing bf16, column copy, quantize, GEMM2"}
+        "note": "GEMM1 4608x3072x21504 + bias (Q, GELU(MLP) -> NVFP4 in the epilogue with the oracle-calibrated "
+                "scale; K,V -> bf16), GEMM2 4608x15360x3072 + bias; unfused = GEMM1 writing bf16, column copy, "
+                "quantize, GEMM2"}
     del y_qm, y_all, y_kv, y2, a2, w1q, w2q, xq, x
     # --- attention-projection sweep, K = N = 3072
     sweep = []
@@ -632,8 +689,15 @@ def run_ours(args):
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
                        "samples": clocks["samples"]},
         }
+        ql_gbs = xl.numel() * QUANT_BYTES_PER_ELEM / (ql_ms * 1e-3) / 1e9
+        line["quantize_roofline"] = {
+            "workload": "laplace_quantize_m4608_k12288", "bound": "hbm", "achieved": ql_gbs, "peak": hbm,
+            "unit": "GB/s", "frac": ql_gbs / hbm, "traffic": quantize_dram_traffic(),
+            "bytes": xl.numel() * QUANT_BYTES_PER_ELEM, "ms": ql_ms,
+            "peak_source": f"{src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src}
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline()
+            line["quantize_cpu_baseline"] = quantize_cpu_baseline()
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

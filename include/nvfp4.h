@@ -36,7 +36,11 @@
  *   - Pointers are device pointers on the current CUDA device, 16-byte
  *     aligned, unless stated otherwise.  The library allocates nothing and
  *     keeps no state besides per-device caches (device properties, the
- *     address of its device fault word).
+ *     address of its device fault word and of its no-allocation scratch,
+ *     each kernel's co-resident grid size).  These caches assume each
+ *     device's primary context lives as long as the process: calls after a
+ *     cudaDeviceReset of a device the library has already used are not
+ *     supported (the cached addresses would be stale).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and is asynchronous: a return of NVFP4_OK means the work was
  *     validated and launched, not that it finished.
@@ -206,6 +210,21 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                         float alpha, const void* bias, void* y, void* stream);
 
 /*
+ * nvfp4_gemm with the two per-tensor scales passed apart, as a ModelOpt layer
+ * stores them (BFL doc, `nvfp4` bullet: `input_scale` and `weight_scale_2`):
+ * the epilogue forms alpha = fl(g_a * g_b) itself (one fp32 product, the same
+ * value a caller computing input_scale * weight_scale_2 in fp32 passes to
+ * nvfp4_gemm).
+ *   g_a  the activation's per-tensor scale (input_scale), finite
+ *   g_b  the weight's per-tensor scale (weight_scale_2), finite
+ *   with g_a * g_b finite.  Other arguments and errors as nvfp4_gemm.
+ */
+nvfp4_status nvfp4_gemm_scaled(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                               const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                               float g_a, float g_b, const void* bias, void* y,
+                               void* stream);
+
+/*
  * nvfp4_gemm for an activation whose per-tensor scale was measured on the
  * device (nvfp4_quantize_dynamic): the epilogue reads g_a from device memory
  * and uses alpha = fl(g_a[0] * g_b) (the same single fp32 product as
@@ -256,6 +275,20 @@ nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_
                               void* y_bf16, int64_t ldy,
                               float g_next, uint8_t* codes_next, uint8_t* sf_next,
                               int64_t k_next, void* stream);
+
+/*
+ * nvfp4_gemm_quant with the two per-tensor scales passed apart (alpha =
+ * fl(g_a * g_b) formed by the epilogue, as in nvfp4_gemm_scaled).  Arguments
+ * and errors as nvfp4_gemm_quant, with g_a, g_b finite and their product
+ * finite in place of alpha.
+ */
+nvfp4_status nvfp4_gemm_quant_scaled(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                     const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                                     float g_a, float g_b, const void* bias,
+                                     const nvfp4_colrange* ranges, int32_t n_ranges,
+                                     void* y_bf16, int64_t ldy,
+                                     float g_next, uint8_t* codes_next, uint8_t* sf_next,
+                                     int64_t k_next, void* stream);
 
 /*
  * ------------------------------------------------------------------------
@@ -365,6 +398,21 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, float g,
  * NVFP4_OK.
  */
 nvfp4_status nvfp4_check_fault(void);
+
+/*
+ * For tests of the failure path only: sets, for the dynamic quantizes
+ * (nvfp4_quantize_dynamic, nvfp4_quantize_dynamic_noalloc) that the calling
+ * host thread launches from now on, how long the kernel's grid-wide wait
+ * lasts (limit_ns; 0 restores the default of one second) and how many
+ * arrivals beyond the grid size it waits for (extra_arrivals; 0 restores the
+ * default).  With extra_arrivals > 0 the wait cannot complete: every CTA gives
+ * up after limit_ns, writes no codes, scales or scale_out, and records
+ * NVFP4_ETIMEOUT in the device fault word (nvfp4_check_fault reports it).  No
+ * other wait and no other entry point is affected.  The pages have no
+ * counterpart; the failure behaviour it exercises is this library's own.
+ * limit_ns <= 10^9, extra_arrivals <= 1024.  Host only.  Errors: EINVAL.
+ */
+nvfp4_status nvfp4_testing_set_grid_wait(uint64_t limit_ns, uint32_t extra_arrivals);
 
 /*
  * Launch shapes the library picks, for callers that size work around them

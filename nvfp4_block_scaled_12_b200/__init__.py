@@ -61,6 +61,10 @@ def _load() -> ctypes.CDLL:
                                      vp, i64, f32, vp, vp, i64, vp]
     lib.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.nvfp4_gemm_dynamic.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp, vp]
+    lib.nvfp4_gemm_scaled.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, f32, vp, vp, vp]
+    lib.nvfp4_gemm_quant_scaled.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, f32, vp, ctypes.POINTER(ColRange),
+                                            i32, vp, i64, f32, vp, vp, i64, vp]
+    lib.nvfp4_testing_set_grid_wait.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
     lib.nvfp4_quantize_dynamic_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp]
     lib.nvfp4_mxfp8_sf_bytes.argtypes = [i64, i64]
     lib.nvfp4_mxfp8_sf_bytes.restype = ctypes.c_size_t
@@ -76,7 +80,8 @@ def _load() -> ctypes.CDLL:
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
                  "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
-                 "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_gemm_tile_shape"):
+                 "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_gemm_tile_shape", "nvfp4_gemm_scaled",
+                 "nvfp4_gemm_quant_scaled", "nvfp4_testing_set_grid_wait"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -133,6 +138,11 @@ def nvfp4_gemm(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha
     _check(library().nvfp4_gemm(a, sfa, b, sfb, M, N, K, alpha, bias or None, y, stream))
 
 
+def nvfp4_gemm_scaled(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_a: float, g_b: float,
+                      bias: int, y: int, stream: int) -> None:
+    _check(library().nvfp4_gemm_scaled(a, sfa, b, sfb, M, N, K, g_a, g_b, bias or None, y, stream))
+
+
 def nvfp4_gemm_dynamic(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_b: float, g_a: int,
                        bias: int, y: int, stream: int) -> None:
     _check(library().nvfp4_gemm_dynamic(a, sfa, b, sfb, M, N, K, g_b, g_a, bias or None, y, stream))
@@ -144,6 +154,19 @@ def nvfp4_gemm_quant(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int,
     arr = (ColRange * len(ranges))(*ranges)
     _check(library().nvfp4_gemm_quant(a, sfa, b, sfb, M, N, K, alpha, bias or None, arr, len(ranges), y_bf16 or None,
                                  ldy, g_next, codes_next or None, sf_next or None, k_next, stream))
+
+
+def nvfp4_gemm_quant_scaled(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_a: float, g_b: float,
+                            bias: int, ranges: Sequence[ColRange], y_bf16: int, ldy: int, g_next: float,
+                            codes_next: int, sf_next: int, k_next: int, stream: int) -> None:
+    arr = (ColRange * len(ranges))(*ranges)
+    _check(library().nvfp4_gemm_quant_scaled(a, sfa, b, sfb, M, N, K, g_a, g_b, bias or None, arr, len(ranges),
+                                             y_bf16 or None, ldy, g_next, codes_next or None, sf_next or None, k_next,
+                                             stream))
+
+
+def nvfp4_testing_set_grid_wait(limit_ns: int, extra_arrivals: int) -> None:
+    _check(library().nvfp4_testing_set_grid_wait(limit_ns, extra_arrivals))
 
 
 def nvfp4_mxfp8_sf_bytes(rows: int, k: int) -> int:
@@ -463,10 +486,11 @@ def swizzle_sf(sf_linear, rows: int, k: int, stream=None):
 
 
 def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = None, y=None, stream=None):
-    """y = bf16(alpha * a_hat @ b_hat^T + bias); alpha defaults to fl32(a.g * b.g)."""
+    """y = bf16(alpha * a_hat @ b_hat^T + bias).  Without ``alpha`` the
+    library forms alpha = fl32(g_a * g_b) from the two per-tensor scales (the
+    activation's read on the device when it was measured there)."""
     torch = _torch()
     dev = torch.cuda.current_device()
-    import numpy as np
     if a.k != b.k:
         raise ValueError("K mismatch")
     M, N, K = a.rows, b.rows, a.k
@@ -474,20 +498,21 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = Non
         raise ValueError("the weight b needs its per-tensor scale g on the host, or pass alpha")
     _need_nvfp4(a, "a", dev=dev)
     _need_nvfp4(b, "b", dev=dev)
-    if alpha is None and a.g is not None:
-        alpha = float(np.float32(a.g) * np.float32(b.g))
     if bias is not None:
         _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
     _need(y, torch.bfloat16, (M, N), "y", dev=dev)
-    if a.g is None and alpha is None:
+    if alpha is not None:
+        nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias),
+                   _ptr(y), _stream(stream))
+    elif a.g is None:
         # the activation's scale lives on the device: alpha = fl32(g_a * g_b) in the kernel
         nvfp4_gemm_dynamic(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(b.g),
                            _ptr(a.scale) + 4, _ptr(bias), _ptr(y), _stream(stream))
-        return y
-    nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias), _ptr(y),
-               _stream(stream))
+    else:
+        nvfp4_gemm_scaled(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(a.g), float(b.g),
+                          _ptr(bias), _ptr(y), _stream(stream))
     return y
 
 
@@ -495,8 +520,8 @@ def gemm_quant(a: NVFP4Tensor, b: NVFP4Tensor, ranges: Sequence[tuple], *, bias=
                g_next: float = 1.0, next_out: Optional[NVFP4Tensor] = None, stream=None) -> None:
     """Fused GEMM whose epilogue writes column ranges to a bf16 tensor and/or
     quantizes them into the next layer's NVFP4 input.  ``ranges`` holds
-    ``(begin, end, act, dst, dst_col)`` tuples."""
-    import numpy as np
+    ``(begin, end, act, dst, dst_col)`` tuples.  Without ``alpha`` the library
+    forms alpha = fl32(g_a * g_b) from the two per-tensor scales."""
     torch = _torch()
     dev = torch.cuda.current_device()
     if a.k != b.k:
@@ -504,10 +529,8 @@ def gemm_quant(a: NVFP4Tensor, b: NVFP4Tensor, ranges: Sequence[tuple], *, bias=
     M, N, K = a.rows, b.rows, a.k
     _need_nvfp4(a, "a", dev=dev)
     _need_nvfp4(b, "b", dev=dev)
-    if alpha is None:
-        if a.g is None or b.g is None:
-            raise ValueError("gemm_quant needs alpha, or both per-tensor scales on the host")
-        alpha = float(np.float32(a.g) * np.float32(b.g))
+    if alpha is None and (a.g is None or b.g is None):
+        raise ValueError("gemm_quant needs alpha, or both per-tensor scales on the host")
     if bias is not None:
         _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
     if y_bf16 is not None:
@@ -524,7 +547,13 @@ def gemm_quant(a: NVFP4Tensor, b: NVFP4Tensor, ranges: Sequence[tuple], *, bias=
     codes_next = next_out.codes if next_out is not None else None
     sf_next = next_out.sf if next_out is not None else None
     k_next = next_out.k if next_out is not None else 0
-    nvfp4_gemm_quant(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias), rs,
-                     _ptr(y_bf16), ldy, float(g_next), _ptr(codes_next), _ptr(sf_next), k_next, _stream(stream))
+    if alpha is not None:
+        nvfp4_gemm_quant(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias),
+                         rs, _ptr(y_bf16), ldy, float(g_next), _ptr(codes_next), _ptr(sf_next), k_next,
+                         _stream(stream))
+    else:
+        nvfp4_gemm_quant_scaled(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(a.g),
+                                float(b.g), _ptr(bias), rs, _ptr(y_bf16), ldy, float(g_next), _ptr(codes_next),
+                                _ptr(sf_next), k_next, _stream(stream))
     if next_out is not None:
         next_out.g = float(g_next)

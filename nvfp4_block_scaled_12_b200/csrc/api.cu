@@ -18,6 +18,10 @@ __device__ unsigned int g_fault_word;
 
 thread_local std::string t_last_error;
 
+// Grid-wait settings the calling thread's dynamic quantizes launch with
+// (changed only by nvfp4_testing_set_grid_wait).
+thread_local GridWaitSettings t_grid_wait;
+
 nvfp4_status fail(nvfp4_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 nvfp4_status fail(nvfp4_status st, const char* fmt, ...) {
   char buf[512];
@@ -40,7 +44,6 @@ nvfp4_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -186,6 +189,11 @@ bool grid_fits(int64_t items, int threads) { return (items + threads - 1) / thre
 
 bool scale_ok(float g) { return finite_f(g) && g >= 0x1p-64f && g <= 0x1p64f; }
 
+// Two per-tensor scales whose fp32 product (the epilogue's alpha) is finite.
+bool product_ok(float g_a, float g_b) {
+  return finite_f(g_a) && finite_f(g_b) && finite_f(static_cast<float>(static_cast<double>(g_a) * g_b));
+}
+
 // Checks shared by the two GEMM entry points; fills the operand part of p
 // and the operand tensor maps.
 // mx: 8-bit operands (one E4M3 byte per element), with E8M0 scales per 32
@@ -223,6 +231,7 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   p->num_kt = static_cast<int32_t>((row_bytes + 127) / 128);
   p->kblocks = static_cast<int32_t>(mx ? K / 32 : K / 64);
   p->alpha = alpha;
+  p->alpha_mul = 1.0f;
   p->bias = static_cast<const __nv_bfloat16*>(bias);
   p->fault = (*dev)->fault;
 
@@ -246,6 +255,81 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   // multiple of 128 may start in the middle of a block
   const uint32_t sfb_blocks = static_cast<uint32_t>(bn % 128 == 0 ? bn / 128 : bn / 128 + 1);
   return make_sf_tmap(&maps->sfb, sfb, N, atoms, box_atoms, sfb_blocks, "B scales");
+}
+
+// nvfp4_gemm_quant with alpha = fl(alpha * alpha_mul) formed on the device.
+nvfp4_status gemm_quant_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                             int64_t M, int64_t N, int64_t K, float alpha, float alpha_mul, const void* bias,
+                             const nvfp4_colrange* ranges, int32_t n_ranges, void* y_bf16, int64_t ldy,
+                             float g_next, uint8_t* codes_next, uint8_t* sf_next, int64_t k_next, void* stream) {
+  if (!ranges || n_ranges < 1 || n_ranges > NVFP4_MAX_RANGES)
+    return fail(NVFP4_EINVAL, "n_ranges=%d must be in [1, %d]", n_ranges, NVFP4_MAX_RANGES);
+  bool any_bf16 = false, any_fp4 = false;
+  for (int i = 0; i < n_ranges; ++i) {
+    const nvfp4_colrange& r = ranges[i];
+    if (r.begin < 0 || r.end <= r.begin || r.end > N || r.begin % 64 || r.end % 64 || r.dst_col < 0 ||
+        r.dst_col % 64)
+      return fail(NVFP4_EINVAL, "range %d [%lld, %lld) -> %lld: bounds must be multiples of 64 within [0, N]", i,
+                  (long long)r.begin, (long long)r.end, (long long)r.dst_col);
+    if (r.act != NVFP4_ACT_NONE && r.act != NVFP4_ACT_GELU_TANH)
+      return fail(NVFP4_EINVAL, "range %d: unknown activation %d", i, r.act);
+    if (r.dst == NVFP4_DST_BF16) {
+      any_bf16 = true;
+      if (r.dst_col + (r.end - r.begin) > ldy) return fail(NVFP4_EINVAL, "range %d overruns ldy", i);
+    } else if (r.dst == NVFP4_DST_NVFP4) {
+      any_fp4 = true;
+      if (r.dst_col + (r.end - r.begin) > k_next) return fail(NVFP4_EINVAL, "range %d overruns k_next", i);
+    } else {
+      return fail(NVFP4_EINVAL, "range %d: unknown destination %d", i, r.dst);
+    }
+    for (int j = 0; j < i; ++j)
+      if (ranges[j].begin < r.end && r.begin < ranges[j].end)
+        return fail(NVFP4_EINVAL, "ranges %d and %d overlap", j, i);
+  }
+  if (any_bf16) {
+    if (!y_bf16) return fail(NVFP4_EINVAL, "a BF16 range needs y_bf16");
+    if (ldy < 8 || ldy % 8 != 0) return fail(NVFP4_EINVAL, "ldy=%lld must be a positive multiple of 8", (long long)ldy);
+    if (!aligned16(y_bf16)) return fail(NVFP4_EALIGN, "y_bf16 must be 16-byte aligned");
+  }
+  if (any_fp4) {
+    if (!codes_next || !sf_next) return fail(NVFP4_EINVAL, "an NVFP4 range needs codes_next and sf_next");
+    if (k_next < 64 || k_next % 64 != 0 || k_next > INT32_MAX / 2)
+      return fail(NVFP4_EINVAL, "k_next=%lld must be a positive multiple of 64", (long long)k_next);
+    if (!scale_ok(g_next)) return fail(NVFP4_EINVAL, "g_next must be finite and in [2^-64, 2^64]");
+    if (!aligned16(codes_next) || !aligned16(sf_next))
+      return fail(NVFP4_EALIGN, "codes_next and sf_next must be 16-byte aligned");
+  }
+  GemmParams p;
+  GemmTensorMaps maps;
+  GemmConfig cg;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev, false, false, true);
+  if (st != NVFP4_OK) return st;
+  if (any_bf16) {
+    st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, ldy, M, ldy * 2, 32, 32,
+                   CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  } else {
+    // never used for a store; a valid descriptor keeps the prefetch harmless
+    st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, 16, 1, 16, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   "dummy");
+  }
+  if (st != NVFP4_OK) return st;
+  p.n_ranges = n_ranges;
+  for (int i = 0; i < n_ranges; ++i) {
+    p.ranges[i].begin = static_cast<int32_t>(ranges[i].begin);
+    p.ranges[i].end = static_cast<int32_t>(ranges[i].end);
+    p.ranges[i].act = ranges[i].act;
+    p.ranges[i].dst = ranges[i].dst;
+    p.ranges[i].dst_col = static_cast<int32_t>(ranges[i].dst_col);
+  }
+  p.g_next = g_next;
+  p.codes_next = codes_next;
+  p.sf_next = sf_next;
+  p.k_next = static_cast<int32_t>(k_next);
+  p.alpha_mul = alpha_mul;
+  cudaError_t e = launch_gemm(maps, p, cg, true, false, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_quant launch");
+  return ok();
 }
 
 }  // namespace
@@ -409,7 +493,7 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t
                  CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
   cudaError_t e = launch_quantize_dynamic(tx, tile_rows, x, M, K, codes, sf, scale_out, static_cast<uint32_t*>(workspace),
-                                          static_cast<cudaStream_t>(stream), *dev);
+                                          t_grid_wait, static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
   return ok();
 }
@@ -438,7 +522,7 @@ nvfp4_status nvfp4_quantize_dynamic_noalloc(const void* x, int64_t M, int64_t K,
                  CU_TENSOR_MAP_SWIZZLE_128B, "x");
   if (st != NVFP4_OK) return st;
   // the launch zeroes the scratch on the stream before the kernel
-  cudaError_t e = launch_quantize_dynamic(tx, tile_rows, x, M, K, codes, sf, scale_out, scratch,
+  cudaError_t e = launch_quantize_dynamic(tx, tile_rows, x, M, K, codes, sf, scale_out, scratch, t_grid_wait,
                                           static_cast<cudaStream_t>(stream), *dev);
   if (e != cudaSuccess) return cuda_fail(e, "dynamic quantize launch");
   return ok();
@@ -476,6 +560,26 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, 
   return ok();
 }
 
+nvfp4_status nvfp4_gemm_scaled(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                               int64_t M, int64_t N, int64_t K, float g_a, float g_b, const void* bias, void* y,
+                               void* stream) {
+  if (!y) return fail(NVFP4_EINVAL, "null output pointer");
+  if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
+  if (!product_ok(g_a, g_b)) return fail(NVFP4_EINVAL, "g_a and g_b must be finite with a finite product");
+  GemmParams p;
+  GemmTensorMaps maps;
+  GemmConfig cg;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev);
+  if (st != NVFP4_OK) return st;
+  p.alpha_mul = g_a;
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm(maps, p, cg, false, false, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return ok();
+}
+
 nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
                                 int64_t M, int64_t N, int64_t K, float g_b, const float* g_a, const void* bias,
                                 void* y, void* stream) {
@@ -496,76 +600,31 @@ nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint
   return ok();
 }
 
+
 nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
                               int64_t M, int64_t N, int64_t K, float alpha, const void* bias,
                               const nvfp4_colrange* ranges, int32_t n_ranges, void* y_bf16, int64_t ldy,
                               float g_next, uint8_t* codes_next, uint8_t* sf_next, int64_t k_next, void* stream) {
-  if (!ranges || n_ranges < 1 || n_ranges > NVFP4_MAX_RANGES)
-    return fail(NVFP4_EINVAL, "n_ranges=%d must be in [1, %d]", n_ranges, NVFP4_MAX_RANGES);
-  bool any_bf16 = false, any_fp4 = false;
-  for (int i = 0; i < n_ranges; ++i) {
-    const nvfp4_colrange& r = ranges[i];
-    if (r.begin < 0 || r.end <= r.begin || r.end > N || r.begin % 64 || r.end % 64 || r.dst_col < 0 ||
-        r.dst_col % 64)
-      return fail(NVFP4_EINVAL, "range %d [%lld, %lld) -> %lld: bounds must be multiples of 64 within [0, N]", i,
-                  (long long)r.begin, (long long)r.end, (long long)r.dst_col);
-    if (r.act != NVFP4_ACT_NONE && r.act != NVFP4_ACT_GELU_TANH)
-      return fail(NVFP4_EINVAL, "range %d: unknown activation %d", i, r.act);
-    if (r.dst == NVFP4_DST_BF16) {
-      any_bf16 = true;
-      if (r.dst_col + (r.end - r.begin) > ldy) return fail(NVFP4_EINVAL, "range %d overruns ldy", i);
-    } else if (r.dst == NVFP4_DST_NVFP4) {
-      any_fp4 = true;
-      if (r.dst_col + (r.end - r.begin) > k_next) return fail(NVFP4_EINVAL, "range %d overruns k_next", i);
-    } else {
-      return fail(NVFP4_EINVAL, "range %d: unknown destination %d", i, r.dst);
-    }
-    for (int j = 0; j < i; ++j)
-      if (ranges[j].begin < r.end && r.begin < ranges[j].end)
-        return fail(NVFP4_EINVAL, "ranges %d and %d overlap", j, i);
-  }
-  if (any_bf16) {
-    if (!y_bf16) return fail(NVFP4_EINVAL, "a BF16 range needs y_bf16");
-    if (ldy < 8 || ldy % 8 != 0) return fail(NVFP4_EINVAL, "ldy=%lld must be a positive multiple of 8", (long long)ldy);
-    if (!aligned16(y_bf16)) return fail(NVFP4_EALIGN, "y_bf16 must be 16-byte aligned");
-  }
-  if (any_fp4) {
-    if (!codes_next || !sf_next) return fail(NVFP4_EINVAL, "an NVFP4 range needs codes_next and sf_next");
-    if (k_next < 64 || k_next % 64 != 0 || k_next > INT32_MAX / 2)
-      return fail(NVFP4_EINVAL, "k_next=%lld must be a positive multiple of 64", (long long)k_next);
-    if (!scale_ok(g_next)) return fail(NVFP4_EINVAL, "g_next must be finite and in [2^-64, 2^64]");
-    if (!aligned16(codes_next) || !aligned16(sf_next))
-      return fail(NVFP4_EALIGN, "codes_next and sf_next must be 16-byte aligned");
-  }
-  GemmParams p;
-  GemmTensorMaps maps;
-  GemmConfig cg;
-  const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev, false, false, true);
-  if (st != NVFP4_OK) return st;
-  if (any_bf16) {
-    st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, ldy, M, ldy * 2, 32, 32,
-                   CU_TENSOR_MAP_SWIZZLE_64B, "Y");
-  } else {
-    // never used for a store; a valid descriptor keeps the prefetch harmless
-    st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, 16, 1, 16, 16, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   "dummy");
-  }
-  if (st != NVFP4_OK) return st;
-  p.n_ranges = n_ranges;
-  for (int i = 0; i < n_ranges; ++i) {
-    p.ranges[i].begin = static_cast<int32_t>(ranges[i].begin);
-    p.ranges[i].end = static_cast<int32_t>(ranges[i].end);
-    p.ranges[i].act = ranges[i].act;
-    p.ranges[i].dst = ranges[i].dst;
-    p.ranges[i].dst_col = static_cast<int32_t>(ranges[i].dst_col);
-  }
-  p.g_next = g_next;
-  p.codes_next = codes_next;
-  p.sf_next = sf_next;
-  p.k_next = static_cast<int32_t>(k_next);
-  cudaError_t e = launch_gemm(maps, p, cg, true, false, static_cast<cudaStream_t>(stream), *dev);
-  if (e != cudaSuccess) return cuda_fail(e, "gemm_quant launch");
+  return gemm_quant_impl(a, sfa, b, sfb, M, N, K, alpha, 1.0f, bias, ranges, n_ranges, y_bf16, ldy, g_next,
+                         codes_next, sf_next, k_next, stream);
+}
+
+nvfp4_status nvfp4_gemm_quant_scaled(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                                     int64_t M, int64_t N, int64_t K, float g_a, float g_b, const void* bias,
+                                     const nvfp4_colrange* ranges, int32_t n_ranges, void* y_bf16, int64_t ldy,
+                                     float g_next, uint8_t* codes_next, uint8_t* sf_next, int64_t k_next,
+                                     void* stream) {
+  if (!product_ok(g_a, g_b)) return fail(NVFP4_EINVAL, "g_a and g_b must be finite with a finite product");
+  return gemm_quant_impl(a, sfa, b, sfb, M, N, K, g_b, g_a, bias, ranges, n_ranges, y_bf16, ldy, g_next,
+                         codes_next, sf_next, k_next, stream);
+}
+
+nvfp4_status nvfp4_testing_set_grid_wait(uint64_t limit_ns, uint32_t extra_arrivals) {
+  if (limit_ns > kWaitLimitNs) return fail(NVFP4_EINVAL, "limit_ns=%llu exceeds the default %llu",
+                                          (unsigned long long)limit_ns, (unsigned long long)kWaitLimitNs);
+  if (extra_arrivals > 1024u) return fail(NVFP4_EINVAL, "extra_arrivals=%u exceeds 1024", extra_arrivals);
+  t_grid_wait.limit_ns = limit_ns == 0 ? kWaitLimitNs : limit_ns;
+  t_grid_wait.extra_arrivals = extra_arrivals;
   return ok();
 }
 

@@ -6,32 +6,10 @@
 // first product is exact in fp32), then rounded to bf16.
 //
 // HBM-bound: 0.5 + 1/16 bytes in, 2 bytes out per element.
-#include <cuda_fp16.h>
-
 #include "internal.h"
 
 namespace nvfp4 {
 namespace {
-
-// Eight E2M1 codes (a 32-bit word, element 2j in the low nibble of byte j)
-// to fp32, exactly: the hardware conversion to f16 pairs, then f16 -> f32.
-__device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float (&f)[8]) {
-  uint32_t h[4];
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(w));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    f[2 * i] = v.x;      // low half: the byte's low nibble
-    f[2 * i + 1] = v.y;
-  }
-}
 
 // One thread per 16 bytes of codes (32 elements, two 16-element blocks):
 // a 16-byte load, the blocks' two scale bytes as one 16-bit load (they are

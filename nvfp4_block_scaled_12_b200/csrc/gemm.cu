@@ -51,6 +51,8 @@
 // Every barrier wait is bounded (see mbar_wait); a role that gives up sets
 // the CTA's abort flag and the device fault word, lets the copies it issued
 // land, and the CTA still reaches the final barrier and frees its TMEM.
+#include <atomic>
+
 #include "internal.h"
 
 namespace nvfp4 {
@@ -66,7 +68,11 @@ constexpr uint32_t kTmemCols = 512;
 // kMx: 8-bit E4M3 operands (K = 32 per MMA) instead of NVFP4; with kRow they
 // carry no block scales at all (row-wise FP8: one scale per row of A and of
 // B, applied in the epilogue), otherwise one E8M0 scale per 32 elements.
-template <int kCG, int kBN, int kAcc, bool kMx, bool kRow = false>
+// kW16: W4A16, bf16 activations (K = 16 per MMA, 64 elements = 128 bytes per
+// k-tile) against NVFP4 weights that the transform warps dequantize to bf16
+// in shared memory (the stage holds this CTA's B codes and scale atoms as
+// loaded, and the bf16 B tile the MMA reads).
+template <int kCG, int kBN, int kAcc, bool kMx, bool kRow = false, bool kW16 = false>
 struct Cfg {
   // Wide tiles (256 columns, one accumulator): the accumulator is drained into
   // the registers of eight epilogue warps, so the next tile's MMAs can start
@@ -79,15 +85,17 @@ struct Cfg {
   // 512-byte scale atoms (128 rows x 4 scale columns) per 128-row block and
   // k-tile: NVFP4's k-tile is 4 MMA k-blocks of 64 elements with one 4-scale
   // word per row each; MXFP8's is 4 k-blocks of 32 whose scales share one word.
-  static constexpr int kAtoms = kMx ? 1 : 4;
-  static constexpr uint32_t kSfaBytes = kRow ? 0 : kAtoms * 512;
+  // (W4A16: a k-tile of 64 elements is one atom, read for B only)
+  static constexpr int kAtoms = (kMx || kW16) ? 1 : 4;
+  static constexpr uint32_t kSfaBytes = (kRow || kW16) ? 0 : kAtoms * 512;
   static constexpr int kBNc = kBN / kCG;  // B rows per CTA
   static constexpr uint32_t kBBytes = kBNc * kBKBytes;
   static constexpr int kChunks = kBN / 32;
   // 128-row scale blocks a B tile can touch (a 192-wide tile may start mid-block)
   static constexpr int kSfbBlocks = kBN % 128 == 0 ? kBN / 128 : kBN / 128 + 1;
   static constexpr uint32_t kSfbBytes = kRow ? 0 : kSfbBlocks * kAtoms * 512;
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr uint32_t kCodeBytes = kW16 ? kBNc * 32 : 0;  // W4A16: this CTA's B codes (64 elements a row)
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kCodeBytes;
   static constexpr uint32_t kEpiBytes = kEpiWarps * 2 * 2048;  // double-buffered 32 x 32 bf16 staging per warp
   static constexpr uint32_t kBiasBytes = kWide ? kEpiWarps * 256 : 0;  // each wide epilogue warp's 128 bias values
   static constexpr int kStagesFit = (224 * 1024 - kEpiBytes - kBiasBytes) / kStageBytes;
@@ -112,14 +120,16 @@ struct Cfg {
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
   static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
   static constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
-  static constexpr uint32_t kOffEpi = kOffSfb + kStages * kSfbBytes;
+  static constexpr uint32_t kOffCode = kOffSfb + kStages * kSfbBytes;
+  static constexpr uint32_t kOffEpi = kOffCode + kStages * kCodeBytes;
   static constexpr uint32_t kOffBias = kOffEpi + kEpiBytes;
   static constexpr uint32_t kOffBar = kOffBias + kBiasBytes;
   // full, empty, sfin per stage; acc_full, acc_empty per accumulator; drain
   static constexpr uint32_t kNumBars = 3 * kStages + 2 * kAcc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t kFullTx = kCG * (kABytes + kBBytes);  // A/B bytes of the whole group
+  // A/B bytes of the whole group (W4A16: A only; B is written by the transform warps)
+  static constexpr uint32_t kFullTx = kW16 ? kCG * kABytes : kCG * (kABytes + kBBytes);
   static_assert(kBN % 32 == 0 && kChunks * 32 == kBN && kBN / kCG % 8 == 0, "tile width");
   static_assert(kBBytes % 1024 == 0, "stage bases must stay 1024-byte aligned");
   static_assert(kSfSlots >= 2 && kSfSlots <= kStages, "TMEM budget");
@@ -128,6 +138,8 @@ struct Cfg {
   static_assert(kStages >= 3 && kStages >= kProducers, "pipeline depth");
   static_assert(!kWide || kCG == 2, "wide tiles are CTA pairs");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(!kW16 || (!kMx && !kRow), "W4A16 has bf16 activations and NVFP4 weights");
+  static_assert(kCodeBytes % 128 == 0 && kSfbBytes % 128 == 0, "TMA destinations stay 128-byte aligned");
 };
 
 __device__ __forceinline__ float gelu_tanh_f32(float v) {
@@ -156,12 +168,13 @@ __device__ __forceinline__ void store_chunk_bf16(const CUtensorMap* tmap, uint8_
   }
 }
 
-template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow>
-__global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
+template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow, bool kW16 = false>
+__global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ GemmParams p) {
-  using C = Cfg<kCG, kBN, kAcc, kMx, kRow>;
+  using C = Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>;
+  static_assert(!(kFused && kW16), "the fused quantize epilogue follows an NVFP4 GEMM");
   static_assert(!(kFused && kMx), "the fused quantize epilogue writes NVFP4 after an NVFP4 GEMM");
   static_assert(!kRow || kMx, "row-wise FP8 uses the 8-bit operand layout");
   constexpr int S = C::kStages;
@@ -171,7 +184,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;            // leader: A/B of the whole group landed, scales in TMEM
   uint64_t* empty = bars + S;       // this CTA's stage and the k-tile's scale slot may be refilled
-  uint64_t* sfin = bars + 2 * S;    // this CTA's scale atoms landed
+  uint64_t* sfin = bars + 2 * S;    // this CTA's scale atoms (W4A16: B codes and scale atoms) landed
   uint64_t* acc_full = bars + 3 * S;
   uint64_t* acc_empty = acc_full + kAcc;   // leader
   uint64_t* drain = acc_empty + kAcc;
@@ -210,10 +223,8 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
-    if (!kRow) {
-      prefetch_tmap(&tmap_sfa);
-      prefetch_tmap(&tmap_sfb);
-    }
+    if (!kRow && !kW16) prefetch_tmap(&tmap_sfa);
+    if (!kRow) prefetch_tmap(&tmap_sfb);
     prefetch_tmap(&tmap_y);
   }
   if (warp == 1) {
@@ -264,18 +275,27 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
         const int n0 = (tile / p.tiles_m) * kBN;
         const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
         if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
-        if (!kRow) mbar_arrive_expect_tx(&sfin[stage], C::kSfaBytes + C::kSfbBytes);
+        if (!kRow) mbar_arrive_expect_tx(&sfin[stage], C::kSfaBytes + C::kSfbBytes + C::kCodeBytes);
         uint8_t* sa = smem + C::kOffA + stage * kABytes;
         uint8_t* sb = smem + C::kOffB + stage * C::kBBytes;
+        // A's x coordinate counts elements of its map: bytes for the 4- and
+        // 8-bit codes, bf16 elements (64 per 128-byte k-tile) for W4A16
+        const int32_t xa = kW16 ? kt * 64 : kt * kBKBytes;
+        const int brow = n0 + static_cast<int>(rank) * C::kBNc;  // this CTA's first B row
         if (kCG == 2) {
           const uint32_t fb = peer_smem(smem_u32(&full[stage]), 0);
-          tma_load_2d_pair(sa, &tmap_a, fb, kt * kBKBytes, row_block * 128);
-          tma_load_2d_pair(sb, &tmap_b, fb, kt * kBKBytes, n0 + static_cast<int>(rank) * C::kBNc);
+          tma_load_2d_pair(sa, &tmap_a, fb, xa, row_block * 128);
+          if (!kW16) tma_load_2d_pair(sb, &tmap_b, fb, kt * kBKBytes, brow);
         } else {
-          tma_load_2d(sa, &tmap_a, &full[stage], kt * kBKBytes, row_block * 128);
-          tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
+          tma_load_2d(sa, &tmap_a, &full[stage], xa, row_block * 128);
+          if (!kW16) tma_load_2d(sb, &tmap_b, &full[stage], kt * kBKBytes, n0);
         }
-        if (!kRow) {
+        if (kW16) {
+          // this CTA's B codes (32 bytes = 64 elements a row) and the B scale
+          // atoms of the k-tile, for the transform warps
+          tma_load_2d(smem + C::kOffCode + stage * C::kCodeBytes, &tmap_b, &sfin[stage], kt * 32, brow);
+          tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt, n0 >> 7);
+        } else if (!kRow) {
           tma_load_3d(smem + C::kOffSfa + stage * C::kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * C::kAtoms, row_block);
           tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * C::kAtoms, n0 >> 7);
         }
@@ -299,7 +319,13 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
       // byte kb of the k-tile's scale words (named in the descriptor and in
       // the top two bits of the scale addresses)
       auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb, int kb, uint32_t accum) {
-        if constexpr (kRow) {
+        if constexpr (kW16) {
+          constexpr uint32_t idesc = idesc_bf16(128 * kCG, kBN);
+          if (kCG == 2)
+            tc_mma_bf16_pair(d, ad, bd, idesc, accum);
+          else
+            tc_mma_bf16(d, ad, bd, idesc, accum);
+        } else if constexpr (kRow) {
           constexpr uint32_t idesc = idesc_f8(128 * kCG, kBN);
           if (kCG == 2)
             tc_mma_f8_pair(d, ad, bd, idesc, accum);
@@ -333,7 +359,9 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          // W4A16 pairs: the peer's transform warps release their B tile at
+          // cluster scope, acquired here before the pair MMA reads it
+          if (!mbar_wait<kW16 && kCG == 2>(&full[stage], phase, abort_flag)) {
             fault = kFaultMmaWait;
             break;
           }
@@ -505,6 +533,71 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     }
     if (fault != 0u) *abort_flag = 1;
   };
+  auto run_transform = [&]() {
+    // ------------------------------------------------------------ W4A16 transform warps
+    // Dequantize this CTA's B rows of each k-tile, as landed (codes 32 bytes
+    // a row, the k-tile's scale atoms), into the stage's bf16 B tile in the
+    // 128-byte-swizzled K-major layout the MMA descriptors describe:
+    //   w = bf16_rn(fl(fl(e2m1(q) * e4m3(s)) * g))   (the first product exact)
+    // Work item i of the 2 * kBNc per k-tile = half i % 2 (32 elements, two
+    // 16-element blocks) of row i / 2; the four warps take every 128th item.
+    if constexpr (kW16) {
+      const int t = (warp & 3) * 32 + lane;
+      const float g = p.alpha_mul;  // the weight's per-tensor scale
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
+        const int n0 = (tile / p.tiles_m) * kBN;
+        const int brow = n0 + static_cast<int>(rank) * C::kBNc;
+        for (int kt = 0; kt < p.num_kt; ++kt) {
+          const bool landed = mbar_wait(&sfin[stage], phase, abort_flag);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, landed)) {
+            fault = kFaultMmaWait;
+            break;
+          }
+          const uint8_t* cb = smem + C::kOffCode + stage * C::kCodeBytes;
+          const uint8_t* sb = smem + C::kOffSfb + stage * C::kSfbBytes;
+          uint8_t* bb = smem + C::kOffB + stage * C::kBBytes;
+#pragma unroll 1
+          for (int i = t; i < 2 * C::kBNc; i += 128) {
+            const int row = i >> 1, half = i & 1;
+            const int rg = brow + row;  // B row in the weight (rows past N arrived zero-filled)
+            const uint4 c = *reinterpret_cast<const uint4*>(cb + row * 32 + half * 16);
+            const int blk = (rg >> 7) - (n0 >> 7);
+            const uint32_t sw = *reinterpret_cast<const uint32_t*>(sb + blk * 512 + (rg & 31) * 16 + ((rg & 127) >> 5) * 4);
+            const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // 8 elements = one 16-byte chunk of bf16
+              const float s = e4m3_to_f32((sw >> (8 * (2 * half + (j >> 1)))) & 0xFFu);
+              float f[8];
+              e2m1x8_to_f32(words[j], f);
+              uint32_t o[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                o[e] = pack_bf16x2(__fmul_rn(__fmul_rn(f[2 * e], s), g), __fmul_rn(__fmul_rn(f[2 * e + 1], s), g));
+              const int chunk = half * 4 + j;
+              *reinterpret_cast<uint4*>(bb + row * 128 + ((chunk ^ (row & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+          // the MMA (async proxy) reads what these generic stores wrote
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (kCG == 2 && !leader)
+              mbar_arrive_cluster_release(peer_smem(smem_u32(&full[stage]), 0));
+            else
+              mbar_arrive(&full[stage]);
+          }
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (fault != 0u) *abort_flag = 1;
+    }
+  };
   // One 32-column chunk of a 32-row slice, as bf16 words (w[j] = columns 2j,
   // 2j+1 of this thread's row): the fused epilogue's column ranges pick the
   // destination and activation; bf16 chunks go out through the TMA, NVFP4
@@ -578,7 +671,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     uint8_t* bias_buf = smem + C::kOffBias + e * 256;
     int buf = 0;
     uint32_t acc_phase = 0;
-    const float alpha = p.alpha_scale != nullptr ? __fmul_rn(p.alpha, *p.alpha_scale) : p.alpha;
+    const float alpha = __fmul_rn(p.alpha, p.alpha_scale != nullptr ? *p.alpha_scale : p.alpha_mul);
     for (int tile = cluster; tile < p.num_tiles; tile += num_clusters) {
       const int tm = tile % p.tiles_m;
       const int c0 = (tile / p.tiles_m) * kBN + h * 128;  // first column of this warp's slice
@@ -656,8 +749,9 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     int buf = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    // alpha = g_a * g_b; with a scale measured on the device, g_a is read here
-    const float alpha = p.alpha_scale != nullptr ? __fmul_rn(p.alpha, *p.alpha_scale) : p.alpha;
+    // alpha = fl(g_a * g_b) when the two scales are passed apart (alpha_mul,
+    // or g_a measured on the device and read here); fl(alpha * 1) = alpha
+    const float alpha = __fmul_rn(p.alpha, p.alpha_scale != nullptr ? *p.alpha_scale : p.alpha_mul);
     for (int tile = cluster; tile < p.num_tiles; tile += num_clusters) {
       const int tm = tile % p.tiles_m;
       const int n0 = (tile / p.tiles_m) * kBN;
@@ -742,7 +836,10 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
         run_mma();
     } else if (wg == 3) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
-      if constexpr (!kRow) run_movers();  // row-wise FP8 has no block scales to move
+      if constexpr (kW16)
+        run_transform();
+      else if constexpr (!kRow)
+        run_movers();  // row-wise FP8 has no block scales to move
     } else {
       asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
       run_epilogue_wide();
@@ -753,7 +850,10 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
     else if (warp == 1)
       run_mma();
     else if (is_mover) {
-      if constexpr (!kRow) run_movers();  // row-wise FP8 has no block scales to move
+      if constexpr (kW16)
+        run_transform();
+      else if constexpr (!kRow)
+        run_movers();  // row-wise FP8 has no block scales to move
     } else if (is_epilogue)
       run_epilogue();
   }
@@ -769,10 +869,10 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow>::kThreads, 1)
   }
 }
 
-template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow = false>
+template <int kCG, int kBN, int kAcc, bool kFused, bool kMx, bool kRow = false, bool kW16 = false>
 cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t stream, const DeviceInfo& dev) {
-  using C = Cfg<kCG, kBN, kAcc, kMx, kRow>;
-  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused, kMx, kRow>;
+  using C = Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>;
+  auto kernel = gemm_nvf4_kernel<kCG, kBN, kAcc, kFused, kMx, kRow, kW16>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -786,8 +886,11 @@ cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t st
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = kCG == 2 ? 1 : 0;
-  // A persistent grid must be co-resident: as many CTA groups as fit at once.
-  static int max_groups = 0;  // per template instance; one device family
+  // A persistent grid must be co-resident: as many CTA groups as fit at once,
+  // found once per template instance and device (two host threads that race
+  // on the first launch compute and store the same value).
+  static std::atomic<int> groups_cache[kMaxDevices];
+  int max_groups = groups_cache[dev.device].load(std::memory_order_relaxed);
   if (max_groups == 0) {
     int n = dev.num_sms / kCG;
     if (kCG == 2) {
@@ -797,6 +900,7 @@ cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t st
         n = clusters;
     }
     max_groups = n;
+    groups_cache[dev.device].store(n, std::memory_order_relaxed);
   }
   const int groups = p.num_tiles < max_groups ? p.num_tiles : max_groups;
   cfg.gridDim = dim3(static_cast<unsigned>(groups * kCG), 1, 1);
@@ -821,6 +925,19 @@ GemmConfig gemm_config(int64_t M, int64_t N, int num_sms) {
   const int64_t tiles128 = ((M + 255) / 256) * ((N + 127) / 128);
   if (tiles192 < pairs && tiles128 <= pairs) return GemmConfig{2, 128, 2};
   return GemmConfig{2, 192, 2};
+}
+
+cudaError_t launch_gemm_w4a16(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, cudaStream_t stream,
+                              const DeviceInfo& dev) {
+  if (c.cta_group == 2 && c.tile_n == 256 && c.acc_bufs == 1)
+    return launch<2, 256, 1, false, false, false, true>(m, p, stream, dev);
+  if (c.cta_group == 2 && c.tile_n == 192 && c.acc_bufs == 2)
+    return launch<2, 192, 2, false, false, false, true>(m, p, stream, dev);
+  if (c.cta_group == 2 && c.tile_n == 128 && c.acc_bufs == 2)
+    return launch<2, 128, 2, false, false, false, true>(m, p, stream, dev);
+  if (c.cta_group == 1 && c.tile_n == 192 && c.acc_bufs == 2)
+    return launch<1, 192, 2, false, false, false, true>(m, p, stream, dev);
+  return cudaErrorInvalidConfiguration;
 }
 
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,

@@ -10,6 +10,9 @@
 
 namespace nvfp4 {
 
+// Devices the per-device caches of the library cover (device index < this).
+constexpr int kMaxDevices = 64;
+
 struct DeviceInfo {
   int device = -1;
   int num_sms = 0;
@@ -29,7 +32,8 @@ struct GemmParams {
   int32_t num_kt;  // k-tiles of 256 elements (last one may be partial)
   int32_t kblocks; // MMA k-blocks in total: K / 64 (NVFP4) or K / 32 (MXFP8)
   float alpha;
-  const float* alpha_scale;   // nullable: if set, the epilogue uses fl(alpha * alpha_scale[0])
+  float alpha_mul;            // the epilogue uses fl(alpha * alpha_mul) (1 when alpha is given whole)
+  const float* alpha_scale;   // nullable: if set, the epilogue uses fl(alpha * alpha_scale[0]) instead
   const float* row_scale;     // row-wise FP8: [M] scales of A's rows
   const float* col_scale;     // row-wise FP8: [N] scales of B's rows (output columns)
   const __nv_bfloat16* bias;  // nullable
@@ -55,6 +59,15 @@ struct DynamicScaleArgs {
   const uint8_t* x;  // bf16 [M, K], for the amax pass
   uint32_t* scratch; // [0] bits of the grid-wide max |x|, [1] CTAs arrived; both start at zero
   float* scale_out;  // [0] amax, [1] g, written by CTA 0
+  uint64_t wait_limit_ns;  // longest wait for the other CTAs' arrivals
+  uint32_t expect;         // arrivals that complete the wait (the grid size, plus any test-only extra)
+};
+
+// Grid-wait settings of the dynamic quantize (normally kWaitLimitNs and no
+// extra arrivals; a test of the time-out path changes them for its thread).
+struct GridWaitSettings {
+  uint64_t limit_ns = kWaitLimitNs;
+  uint32_t extra_arrivals = 0;
 };
 // Bytes of scratch one dynamic-scale quantize uses (zeroed by the launch).
 constexpr size_t kDynamicScratchBytes = 8;
@@ -71,7 +84,7 @@ cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int tile_rows, int6
 // Same, with g measured on x in the same (cooperative) launch.
 cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, int tile_rows, const void* x, int64_t M, int64_t K,
                                     uint8_t* codes, uint8_t* sf, float* scale_out, uint32_t* scratch,
-                                    cudaStream_t stream, const DeviceInfo& dev);
+                                    const GridWaitSettings& wait, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_calibrate(const void* x, int64_t n, float* out, cudaStream_t stream, const DeviceInfo& dev);
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out, cudaStream_t stream);
 
@@ -86,6 +99,12 @@ GemmConfig gemm_config(int64_t M, int64_t N, int num_sms);
 // row: row-wise FP8 (8-bit operands without block scales; requires mx).
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
                         cudaStream_t stream, const DeviceInfo& dev, bool row = false);
+// W4A16: bf16 activations [M, K] x NVFP4 weights [N, K] dequantized in shared
+// memory (p.alpha_mul carries the weight's per-tensor scale, p.alpha = 1);
+// maps: a = bf16 activations (64-element boxes), b = weight codes (32-byte
+// boxes of this CTA's B rows), sfb = weight scales (one atom per k-tile).
+cudaError_t launch_gemm_w4a16(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, cudaStream_t stream,
+                              const DeviceInfo& dev);
 // NVFP4 [rows, K] (codes, swizzled scales, g) -> bf16 [rows, K].
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* sf, float g, int64_t rows, int64_t K, void* out,
                               cudaStream_t stream);

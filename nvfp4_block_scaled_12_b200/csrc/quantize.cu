@@ -23,7 +23,9 @@
 // then starts the TMA ring at once (the tiles do not depend on the scale)
 // while the consumers wait for the counter to reach the grid size, so the
 // second read of a tile usually comes from L2.  The grid is launched
-// cooperatively (every CTA resident), and the wait is bounded.
+// cooperatively (every CTA resident), and the wait is bounded (by default
+// kWaitLimitNs; a test of the time-out path shortens it and adds arrivals that
+// never come, see nvfp4_testing_set_grid_wait).
 #include "internal.h"
 
 namespace nvfp4 {
@@ -107,14 +109,15 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
         tma_load_2d(smem + stage * Q::kTileBytes, &tmap_x, &full[stage], static_cast<int32_t>((tile % tiles_k) * Q::kCols),
                     static_cast<int32_t>((tile / tiles_k) * Q::kTileRows));
       }
-      if (fault != 0u) {
-        *abort_flag = 1;
-        // let the copies already issued (the last Q::kStages entries) land
-        for (int64_t k = jj - 1; k >= 0 && k >= jj - Q::kStages; --k) {
-          const int64_t i = k / Q::kGroups;
-          const int stage = static_cast<int>(k % Q::kGroups) * Q::kStagesPerGroup + static_cast<int>(i % Q::kStagesPerGroup);
-          mbar_wait(&full[stage], static_cast<uint32_t>((i / Q::kStagesPerGroup) & 1), nullptr);
-        }
+      if (fault != 0u) *abort_flag = 1;
+      // Every copy this warp issued (the last Q::kStages entries at most) has
+      // landed before the CTA may exit, also when the consumers gave up before
+      // taking them (normally they have taken them all and these waits return
+      // at once).
+      for (int64_t k = jj - 1; k >= 0 && k >= jj - Q::kStages; --k) {
+        const int64_t i = k / Q::kGroups;
+        const int stage = static_cast<int>(k % Q::kGroups) * Q::kStagesPerGroup + static_cast<int>(i % Q::kStagesPerGroup);
+        mbar_wait(&full[stage], static_cast<uint32_t>((i / Q::kStagesPerGroup) & 1), nullptr);
       }
     }
   } else {
@@ -151,11 +154,11 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
         atomicAdd(dyn.scratch + 1, 1u);
         const uint64_t t0 = global_timer_ns();
         uint32_t arrived;
-        while ((arrived = ld_acquire_gpu(dyn.scratch + 1)) < gridDim.x) {
-          if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) break;
+        while ((arrived = ld_acquire_gpu(dyn.scratch + 1)) < dyn.expect) {
+          if (*abort_flag || global_timer_ns() - t0 > dyn.wait_limit_ns) break;
           __nanosleep(64);
         }
-        warp_max[Q::kConsumerWarps] = arrived >= gridDim.x ? __uint_as_float(ld_acquire_gpu(dyn.scratch)) : -1.0f;
+        warp_max[Q::kConsumerWarps] = arrived >= dyn.expect ? __uint_as_float(ld_acquire_gpu(dyn.scratch)) : -1.0f;
       }
       named_barrier_sync(1, Q::kConsumerWarps * 32);
       const float amax = warp_max[Q::kConsumerWarps];
@@ -343,7 +346,8 @@ namespace {
 
 template <bool kDynamic, bool kMx, int kRows>
 cudaError_t launch_q(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_t K, float g, uint8_t* codes,
-                     uint8_t* sf, float* scale_out, uint32_t* scratch, cudaStream_t stream, const DeviceInfo& dev) {
+                     uint8_t* sf, float* scale_out, uint32_t* scratch, const GridWaitSettings& wait,
+                     cudaStream_t stream, const DeviceInfo& dev) {
   using Q = QCfg<kRows>;
   const int64_t tiles_m = (M + kRows - 1) / kRows;
   const int64_t tiles_k = (K + Q::kCols - 1) / Q::kCols;
@@ -370,7 +374,8 @@ cudaError_t launch_q(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const DynamicScaleArgs dyn{static_cast<const uint8_t*>(x), scratch, scale_out};
+  const DynamicScaleArgs dyn{static_cast<const uint8_t*>(x), scratch, scale_out, wait.limit_ns,
+                             static_cast<uint32_t>(grid) + wait.extra_arrivals};
   err = cudaLaunchKernelEx(&cfg, kernel, tmap_x, M, K, 0.0f, codes, sf, tiles_k, n_tiles, dev.fault, dyn);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
@@ -380,22 +385,24 @@ cudaError_t launch_q(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_
 
 cudaError_t launch_quantize(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, float g, uint8_t* codes,
                             uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev) {
-  return tile_rows == 256 ? launch_q<false, false, 256>(tmap_x, nullptr, M, K, g, codes, sf, nullptr, nullptr, stream, dev)
-                          : launch_q<false, false, 128>(tmap_x, nullptr, M, K, g, codes, sf, nullptr, nullptr, stream, dev);
+  const GridWaitSettings none;
+  return tile_rows == 256 ? launch_q<false, false, 256>(tmap_x, nullptr, M, K, g, codes, sf, nullptr, nullptr, none, stream, dev)
+                          : launch_q<false, false, 128>(tmap_x, nullptr, M, K, g, codes, sf, nullptr, nullptr, none, stream, dev);
 }
 
 cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, uint8_t* codes,
                                   uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev) {
-  return tile_rows == 256 ? launch_q<false, true, 256>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, stream, dev)
-                          : launch_q<false, true, 128>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, stream, dev);
+  const GridWaitSettings none;
+  return tile_rows == 256 ? launch_q<false, true, 256>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, none, stream, dev)
+                          : launch_q<false, true, 128>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, none, stream, dev);
 }
 
 cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, int tile_rows, const void* x, int64_t M, int64_t K,
                                     uint8_t* codes, uint8_t* sf, float* scale_out, uint32_t* scratch,
-                                    cudaStream_t stream, const DeviceInfo& dev) {
+                                    const GridWaitSettings& wait, cudaStream_t stream, const DeviceInfo& dev) {
   return tile_rows == 256
-             ? launch_q<true, false, 256>(tmap_x, x, M, K, 0.0f, codes, sf, scale_out, scratch, stream, dev)
-             : launch_q<true, false, 128>(tmap_x, x, M, K, 0.0f, codes, sf, scale_out, scratch, stream, dev);
+             ? launch_q<true, false, 256>(tmap_x, x, M, K, 0.0f, codes, sf, scale_out, scratch, wait, stream, dev)
+             : launch_q<true, false, 128>(tmap_x, x, M, K, 0.0f, codes, sf, scale_out, scratch, wait, stream, dev);
 }
 
 cudaError_t launch_swizzle_sf(const uint8_t* sf_lin, int64_t rows, int64_t k, uint8_t* out,

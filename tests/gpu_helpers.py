@@ -40,3 +40,14 @@ def assert_within_tol(y_gpu: np.ndarray, y_ref: np.ndarray, tol: np.ndarray, wha
     bad = np.argwhere(~(err <= tol))
     assert bad.size == 0, (f"{what}: {len(bad)} of {err.size} outside tolerance; first {bad[:5].tolist()}: "
                            f"got {y_gpu[tuple(bad[0])]} want {y_ref[tuple(bad[0])]} tol {tol[tuple(bad[0])]}")
+
+
+def single_stream_scales() -> dict:
+    """Per-tensor scales of the FLUX single-stream block pair, written by
+    tests/golden/make_golden.py from the oracle alone: the output
+    projection's calibrated input scale is ``g_next``."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "single_stream_pair.json")
+    with open(path) as f:
+        return json.load(f)

@@ -168,3 +168,22 @@ def test_valid_arguments_without_a_device_fail_loudly_not_silently():
     with pytest.raises(F.NVFP4Error) as e:
         F.nvfp4_quantize(P, 4, 64, 1.0, P, P, 0)
     assert e.value.status in (F.NVFP4_ECUDA, F.NVFP4_EARCH)
+
+
+def test_scaled_gemms_reject_bad_scales_on_the_host():
+    # the two per-tensor scales must be finite and so must their fp32 product
+    for ga, gb in ((float("nan"), 1.0), (1.0, float("inf")), (2.0 ** 100, 2.0 ** 100)):
+        _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_scaled, P, P, P, P, 16, 64, 64, ga, gb, 0, P, 0)
+        rs = [F.ColRange(0, 64, F.ACT_NONE, F.DST_NVFP4, 0)]
+        _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_quant_scaled, P, P, P, P, 16, 64, 64, ga, gb, 0, rs, 0, 0, 0.1, P, P,
+                64, 0)
+    # sizes and alignment are checked as for nvfp4_gemm
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_scaled, P, P, P, P, 16, 12, 64, 1.0, 1.0, 0, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_gemm_scaled, P, P, P, P, 16, 64, 64, 1.0, 1.0, 0, P + 4, 0)
+
+
+def test_grid_wait_knob_checks_its_limits_and_resets():
+    _expect(F.NVFP4_EINVAL, F.nvfp4_testing_set_grid_wait, 2 * 10 ** 9, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_testing_set_grid_wait, 1000, 5000)
+    F.nvfp4_testing_set_grid_wait(1000, 1)
+    F.nvfp4_testing_set_grid_wait(0, 0)  # back to the defaults

@@ -37,7 +37,7 @@ def empty(*shape, dtype=torch.uint8, dev=0):
 def calls(monkeypatch):
     rec = []
     for name in ("nvfp4_quantize", "nvfp4_quantize_dynamic", "nvfp4_gemm", "nvfp4_gemm_dynamic",
-                 "nvfp4_gemm_quant", "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize",
+                 "nvfp4_gemm_scaled", "nvfp4_gemm_quant_scaled", "nvfp4_gemm_quant", "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize",
                  "nvfp4_fp8row_gemm", "nvfp4_dequantize"):
         monkeypatch.setattr(F, name, lambda *a, _n=name: rec.append(_n))
     monkeypatch.setattr(F, "_stream", lambda stream: 0)
@@ -71,8 +71,8 @@ def test_well_formed_buffers_reach_the_library(calls):
     rw = F.FP8RowTensor(empty(N, K), empty(N, dtype=torch.float32), N, K)
     F.quantize_fp8row(x, out=r8)
     F.gemm_fp8row(r8, rw, y=y)
-    assert calls == ["nvfp4_quantize", "nvfp4_gemm", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic",
-                     "nvfp4_gemm_quant", "nvfp4_dequantize", "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm",
+    assert calls == ["nvfp4_quantize", "nvfp4_gemm_scaled", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic",
+                     "nvfp4_gemm_quant_scaled", "nvfp4_dequantize", "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm",
                      "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm"]
 
 

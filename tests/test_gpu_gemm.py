@@ -66,7 +66,8 @@ def test_tiny_workload(F):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 8, 64), (100, 200, 192), (129, 392, 320), (300, 64, 1024),
-                                   (128, 192, 256), (256, 384, 512), (77, 1000, 4096), (1000, 3000, 1088)])
+                                   (128, 192, 256), (256, 384, 512), (77, 1000, 4096), (1000, 3000, 1088),
+                                   (300, 520, 15360), (97, 136, 15424)])
 def test_ragged_shapes(F, m, n, k):
     _check_linear(F, synth.LinearWorkload(f"ragged_{m}x{n}x{k}", m, k, n, seed=m + n + k))
 
@@ -74,6 +75,23 @@ def test_ragged_shapes(F, m, n, k):
 @pytest.mark.parametrize("idx", [0, 1])
 def test_sweep_small_token_counts_full(F, idx):
     _check_linear(F, synth.SWEEP[idx])
+
+
+@pytest.mark.parametrize("idx", [2, 3, 4])
+def test_sweep_large_token_counts_sampled(F, idx):
+    # The token sweep's larger points (M = 4608, 9216, 16896; K = N = 3072):
+    # all columns of sampled rows (the last ones included) and all rows of
+    # sampled columns.
+    wl = synth.SWEEP[idx]
+    rng = np.random.default_rng(wl.seed)
+    rows = np.unique(np.r_[rng.choice(wl.m, 64, replace=False), wl.m - 1, wl.m - 129, 255, 256])
+    y = _check_linear(F, wl, rows=rows)
+    x, w, b = wl.activations(), wl.weight(), wl.bias_vec()
+    (xc, xs, gx), (wc, ws, gw) = _oracle_layer(x, w)
+    cols = np.unique(np.r_[rng.choice(wl.n, 48, replace=False), wl.n - 1, 255, 256])
+    y_ref = O.gemm_ref(xc, xs, gx, wc[cols], ws[cols], gw, b.float().numpy()[cols])
+    tol = O.gemm_tolerance(xc, xs, gx, wc[cols], ws[cols], gw, y_ref)
+    assert_within_tol(y[:, cols], y_ref, tol, wl.name + " columns")
 
 
 def test_mlp_up_full_size_sampled(F):
@@ -168,7 +186,8 @@ def _wide(M, N):
     return F.nvfp4_gemm_tile_shape(M, N, sms) == (2, 256, 1)
 
 
-@pytest.mark.parametrize("m,n,k", [(2341, 2056, 3136), (4608, 3072, 3072), (2305, 8200, 1088)])
+@pytest.mark.parametrize("m,n,k", [(2341, 2056, 3136), (4608, 3072, 3072), (2305, 8200, 1088),
+                                   (2341, 2056, 15360)])
 def test_wide_tiles_ragged_sampled(F, m, n, k):
     # Shapes that take the 256 x 256 tiles, ragged in M, N and K (a last
     # k-tile with one or two MMA k-blocks): all columns of sampled rows (the

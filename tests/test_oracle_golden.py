@@ -51,3 +51,20 @@ def test_tiny_workload_regression_fixture():
     y = O.gemm_ref(xc, xs, gx, wc, ws, gw)
     assert abs(y[0, 0] - want["y_00"]) < 1e-12 and abs(y[-1, -1] - want["y_last"]) < 1e-12
     assert abs(y.sum() - want["y_sum"]) < 1e-9
+
+
+def test_single_stream_pair_fixture_matches_the_oracle():
+    # The stored scales of the single-stream pair (written by make_golden.py,
+    # which calls only the oracle and the input generators): recomputed here,
+    # including the output projection's calibrated input scale from the
+    # oracle's full GEMM1 and fused epilogue.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(GOLDEN, "make_golden.py"))
+    MG = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(MG)
+    with open(os.path.join(GOLDEN, "single_stream_pair.json")) as f:
+        fx = json.load(f)
+    got = MG.single_stream_pair()
+    for key in ("g_x", "g_w1", "g_w2", "amax_next", "g_next"):
+        assert np.float32(got[key]) == np.float32(fx[key]), key
+    assert np.float32(fx["g_next"]) == O.global_scale(np.float32(fx["amax_next"]))

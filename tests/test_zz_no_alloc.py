@@ -1,17 +1,19 @@
 """The no-allocation dynamic quantize, nvfp4_quantize_dynamic_noalloc, against
-the workspace entry point nvfp4_quantize_dynamic, both called through the C
-ABI with raw device pointers.  Two calls in a row (on tensors with different
-scales, so the shared scratch must be re-zeroed by each call) must give the
-same codes, scales, amax and g as the workspace path.  This file sorts last
-so that it also runs after every other GPU test in one session; it passes
+the workspace entry point nvfp4_quantize_dynamic and against the oracle, all
+called through the C ABI with raw device pointers.  Two calls in a row (on
+tensors with different scales, so the shared scratch must be re-zeroed by each
+call) must give the same codes, scales, amax and g as the workspace path, and
+both must equal the oracle's dynamic quantize bit for bit.  This file sorts
+last so that it also runs after every other GPU test in one session; it passes
 alone as well.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import synth
-from tests.gpu_helpers import assert_bytes_equal, gpu_bytes, require_gpu
+from tests.gpu_helpers import assert_bytes_equal, f32, gpu_bytes, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +61,11 @@ def test_no_alloc_matches_the_workspace_entry_point_twice_in_a_row(F):
         assert_bytes_equal(gpu_bytes(got[0]), gpu_bytes(want[0]), "no-alloc codes")
         assert_bytes_equal(gpu_bytes(got[1]), gpu_bytes(want[1]), "no-alloc scales")
         assert np.array_equal(got[2].cpu().numpy(), want[2].cpu().numpy())
+        # and the oracle's dynamic quantize of the same bf16 values
+        codes, sf, amax, g = O.quantize_dynamic(f32(x.cpu()))
+        assert_bytes_equal(gpu_bytes(got[0]), codes, "no-alloc codes vs oracle")
+        assert_bytes_equal(gpu_bytes(got[1]), O.swizzle_sf(sf), "no-alloc scales vs oracle")
+        assert np.array_equal(got[2].cpu().numpy(), np.array([amax, g], np.float32))
     F.nvfp4_check_fault()
 
 
