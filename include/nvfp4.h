@@ -382,14 +382,35 @@ nvfp4_status nvfp4_fp8row_gemm(const uint8_t* a, const float* a_scale, const uin
  * forward and the layer runs as a regular linear with bf16 activations):
  * NVFP4 -> bf16,
  *     out[r, k] = bf16_rn( fl( fl(e2m1(code) * e4m3(scale)) * g ) )
- * (the first product is exact in fp32).  The linear itself is a plain bf16
- * GEMM (a library GEMM), not part of this library.
+ * (the first product is exact in fp32).  nvfp4_w4a16_gemm runs the whole
+ * layer without storing these values; this call materializes them.
  *   codes [rows, K/2], sf swizzled nvfp4_sf_bytes(rows, K), g finite;
  *   out   [rows, K] bf16, written.
  * rows >= 1, K % 64 == 0.  Errors: EINVAL, EALIGN, EARCH, ECUDA.
  */
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* sf, float g,
                               int64_t rows, int64_t K, void* out, void* stream);
+
+/*
+ * W4A16 linear layer in one kernel (BFL doc, "Kernels", last paragraph: the
+ * NVFP4 weights dequantized to the compute dtype, the activations left in
+ * bf16, a regular linear):
+ *     y[m, n] = bf16_rn( sum_k x[m, k] * w[n, k] + bias[n] )
+ *     w[n, k] = bf16_rn( fl( fl(e2m1(code) * e4m3(scale)) * g_w ) )
+ * -- exactly the values nvfp4_dequantize writes, formed tile by tile in shared
+ * memory and never stored -- with the sum accumulated in fp32 by the tensor
+ * cores (tcgen05, kind::f16, bf16 x bf16).
+ *   x        [M, K] bf16 activations
+ *   w_codes  [N, K/2] NVFP4 weight codes, w_sf swizzled nvfp4_sf_bytes(N, K),
+ *   g_w      the weight's per-tensor scale (weight_scale_2), finite
+ *   bias     [N] bf16 or NULL;  y  [M, N] bf16, written
+ * M >= 1, N >= 8 with N % 8 == 0, K % 64 == 0; the same tile shapes as
+ * nvfp4_gemm.  Errors: EINVAL, EALIGN, EARCH, ECUDA; a barrier time-out
+ * records NVFP4_ETIMEOUT (nvfp4_check_fault).
+ */
+nvfp4_status nvfp4_w4a16_gemm(const void* x, const uint8_t* w_codes, const uint8_t* w_sf,
+                              int64_t M, int64_t N, int64_t K, float g_w, const void* bias,
+                              void* y, void* stream);
 
 /*
  * Synchronize the current device, then read and clear its fault word.

@@ -73,6 +73,7 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_fp8row_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
     lib.nvfp4_fp8row_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
     lib.nvfp4_dequantize.argtypes = [vp, vp, f32, i64, i64, vp, vp]
+    lib.nvfp4_w4a16_gemm.argtypes = [vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
     lib.nvfp4_gemm_tile_shape.argtypes = [i64, i64, i32, ctypes.POINTER(ctypes.c_int32)]
     lib.nvfp4_quantize_tile_rows.argtypes = [i64, i64, i32]
@@ -81,7 +82,7 @@ def _load() -> ctypes.CDLL:
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
                  "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
                  "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_gemm_tile_shape", "nvfp4_gemm_scaled",
-                 "nvfp4_gemm_quant_scaled", "nvfp4_testing_set_grid_wait"):
+                 "nvfp4_gemm_quant_scaled", "nvfp4_testing_set_grid_wait", "nvfp4_w4a16_gemm"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -193,6 +194,11 @@ def nvfp4_fp8row_gemm(a: int, a_scale: int, b: int, b_scale: int, M: int, N: int
 
 def nvfp4_dequantize(codes: int, sf: int, g: float, rows: int, K: int, out: int, stream: int) -> None:
     _check(library().nvfp4_dequantize(codes, sf, g, rows, K, out, stream))
+
+
+def nvfp4_w4a16_gemm(x: int, w_codes: int, w_sf: int, M: int, N: int, K: int, g_w: float, bias: int, y: int,
+                     stream: int) -> None:
+    _check(library().nvfp4_w4a16_gemm(x, w_codes, w_sf, M, N, K, g_w, bias or None, y, stream))
 
 
 def nvfp4_check_fault() -> None:
@@ -466,13 +472,27 @@ def dequantize(t: NVFP4Tensor, out=None, stream=None):
     return out
 
 
-def linear_w4a16(x, w: NVFP4Tensor, bias=None, w_bf16=None, stream=None):
-    """W4A16 linear: the NVFP4 weight dequantized to bf16 by this library,
-    then a regular bf16 linear (a library GEMM) on the unquantized
-    activations."""
+def linear_w4a16(x, w: NVFP4Tensor, bias=None, y=None, stream=None):
+    """W4A16 linear y = bf16(x @ w_bf16^T + bias): bf16 activations ``x``
+    [M, K] against an NVFP4 weight that the GEMM dequantizes tile by tile in
+    shared memory (the values ``dequantize`` would write), in one kernel."""
     torch = _torch()
-    w_bf16 = dequantize(w, out=w_bf16, stream=stream)
-    return torch.nn.functional.linear(x, w_bf16, bias)
+    dev = torch.cuda.current_device()
+    if w.g is None:
+        raise ValueError("the weight needs its per-tensor scale g on the host")
+    M, K = x.shape
+    N = w.rows
+    if w.k != K:
+        raise ValueError("K mismatch")
+    _need(x, torch.bfloat16, None, "x", dev=dev)
+    _need_nvfp4(w, "w", dev=dev)
+    if bias is not None:
+        _need(bias, torch.bfloat16, (N,), "bias", dev=dev)
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _need(y, torch.bfloat16, (M, N), "y", dev=dev)
+    nvfp4_w4a16_gemm(_ptr(x), _ptr(w.codes), _ptr(w.sf), M, N, K, float(w.g), _ptr(bias), _ptr(y), _stream(stream))
+    return y
 
 
 def swizzle_sf(sf_linear, rows: int, k: int, stream=None):

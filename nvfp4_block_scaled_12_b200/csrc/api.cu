@@ -580,6 +580,55 @@ nvfp4_status nvfp4_gemm_scaled(const uint8_t* a, const uint8_t* sfa, const uint8
   return ok();
 }
 
+nvfp4_status nvfp4_w4a16_gemm(const void* x, const uint8_t* w_codes, const uint8_t* w_sf, int64_t M, int64_t N,
+                              int64_t K, float g_w, const void* bias, void* y, void* stream) {
+  if (!x || !w_codes || !w_sf || !y) return fail(NVFP4_EINVAL, "null pointer");
+  nvfp4_status st = check_rows_k("M", M, "K", K);
+  if (st != NVFP4_OK) return st;
+  if (N < 8 || N % 8 != 0 || N > kMaxDim)
+    return fail(NVFP4_EINVAL, "N=%lld must be a positive multiple of 8, at most %lld", (long long)N,
+                (long long)kMaxDim);
+  if (!finite_f(g_w)) return fail(NVFP4_EINVAL, "g_w must be finite");
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(bias) || !aligned16(y))
+    return fail(NVFP4_EALIGN, "pointers must be 16-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  const GemmConfig cg = gemm_config(M, N, dev->num_sms);
+  GemmParams p{};
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(N);
+  p.K = static_cast<int32_t>(K);
+  p.tiles_m = static_cast<int32_t>((M + 128 * cg.cta_group - 1) / (128 * cg.cta_group));
+  p.tiles_n = static_cast<int32_t>((N + cg.tile_n - 1) / cg.tile_n);
+  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  if (tiles > INT32_MAX) return fail(NVFP4_EINVAL, "problem too large");
+  p.num_tiles = static_cast<int32_t>(tiles);
+  p.num_kt = static_cast<int32_t>(K / 64);    // 64 bf16 elements = 128 bytes of every A row
+  p.kblocks = static_cast<int32_t>(K / 16);   // K = 16 per MMA
+  p.alpha = 1.0f;
+  p.alpha_mul = 1.0f;
+  p.w_scale = g_w;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.fault = dev->fault;
+  GemmTensorMaps maps;
+  st = make_tmap(&maps.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+                 "x");
+  if (st != NVFP4_OK) return st;
+  st = make_tmap(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 32,
+                 static_cast<uint32_t>(cg.tile_n / cg.cta_group), CU_TENSOR_MAP_SWIZZLE_NONE, "weight codes");
+  if (st != NVFP4_OK) return st;
+  maps.sfa = maps.b;  // unused (the activations carry no block scales); a valid descriptor
+  const uint32_t sfb_blocks = static_cast<uint32_t>(cg.tile_n % 128 == 0 ? cg.tile_n / 128 : cg.tile_n / 128 + 1);
+  st = make_sf_tmap(&maps.sfb, w_sf, N, K / 64, 1, sfb_blocks, "weight scales");
+  if (st != NVFP4_OK) return st;
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm_w4a16(maps, p, cg, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16 gemm launch");
+  return ok();
+}
+
 nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
                                 int64_t M, int64_t N, int64_t K, float g_b, const float* g_a, const void* bias,
                                 void* y, void* stream) {

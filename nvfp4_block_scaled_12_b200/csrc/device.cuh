@@ -115,6 +115,14 @@ __device__ __forceinline__ uint32_t quantize_mx_block32(const float (&v)[32], ui
   return static_cast<uint32_t>(s + 127);
 }
 
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // Eight E2M1 codes (a 32-bit word, element 2j in the low nibble of byte j)
 // to fp32, exactly: the hardware conversion to f16 pairs, then f16 -> f32.
 __device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float (&f)[8]) {
@@ -135,18 +143,53 @@ __device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float (&f)[8]) {
   }
 }
 
+// Two E4M3 bytes (bits 0-7 and 8-15 of b) to an f16 pair, exactly (E4M3's
+// whole range, subnormals included, is representable in f16); the low byte
+// lands in the low half.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t b) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(b));
+  return h;
+}
+
+// Eight NVFP4 weight elements (a 32-bit word of E2M1 codes, element 2j in the
+// low nibble of byte j) of one 16-element block with E4M3 scale s, to eight
+// bf16 values (four words, element 2j in the low half of word j):
+//     w = bf16_rn( fl32( fl32(e2m1 * s) * g ) )
+// s2 holds s in both halves of an f16 pair.  e2m1 * s has at most six
+// significant bits and lies in [2^-10, 2688], so the f16 product is exact
+// (as it is in fp32); the multiply by g is one fp32 rounding per element,
+// done two at a time (mul.rn.f32x2), then one bf16 rounding.
+__device__ __forceinline__ void nvfp4x8_to_bf16(uint32_t codes, uint32_t s2, float g, uint32_t (&o)[4]) {
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(codes));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t t;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(h[i]), "r"(s2));  // exact
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&t));
+    float lo, hi;
+    asm("{\n\t.reg .b64 a, gg;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 gg, {%4, %4};\n\t"
+        "mul.rn.f32x2 a, a, gg;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "=f"(lo), "=f"(hi) : "f"(f.x), "f"(f.y), "f"(g));
+    o[i] = pack_bf16x2(lo, hi);
+  }
+}
+
 // Byte offset of logical scale (row r, scale column c) in the swizzled
 // scale-factor buffer with `katoms` 4-column atoms per 128-row block.
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t katoms) {
   return ((r >> 7) * katoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // ---------------------------------------------------------------------------
@@ -271,13 +314,6 @@ __device__ __forceinline__ uint32_t peer_smem(uint32_t local, uint32_t rank) {
 // and a cluster-scope release costs hundreds of nanoseconds per arrive.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-// mbar_arrive_cluster with release semantics at cluster scope: for data a
-// thread of one CTA wrote to its own shared memory that work issued from the
-// other CTA of the pair reads (the pair MMA reads both CTAs' operand tiles).
-__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // All threads of both CTAs of the cluster.

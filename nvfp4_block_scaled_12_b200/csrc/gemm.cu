@@ -359,9 +359,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kt = 0; kt < p.num_kt; ++kt) {
-          // W4A16 pairs: the peer's transform warps release their B tile at
-          // cluster scope, acquired here before the pair MMA reads it
-          if (!mbar_wait<kW16 && kCG == 2>(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
             fault = kFaultMmaWait;
             break;
           }
@@ -543,7 +541,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
     // 16-element blocks) of row i / 2; the four warps take every 128th item.
     if constexpr (kW16) {
       const int t = (warp & 3) * 32 + lane;
-      const float g = p.alpha_mul;  // the weight's per-tensor scale
+      const float g = p.w_scale;  // the weight's per-tensor scale
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
@@ -567,28 +565,26 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
             const int blk = (rg >> 7) - (n0 >> 7);
             const uint32_t sw = *reinterpret_cast<const uint32_t*>(sb + blk * 512 + (rg & 31) * 16 + ((rg & 127) >> 5) * 4);
             const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+            // this half's two block scales as an f16 pair (low half: the first block)
+            const uint32_t s01 = e4m3x2_to_f16x2(sw >> (16 * half));
+            const uint32_t sb0 = __byte_perm(s01, 0u, 0x1010), sb1 = __byte_perm(s01, 0u, 0x3232);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {  // 8 elements = one 16-byte chunk of bf16
-              const float s = e4m3_to_f32((sw >> (8 * (2 * half + (j >> 1)))) & 0xFFu);
-              float f[8];
-              e2m1x8_to_f32(words[j], f);
               uint32_t o[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                o[e] = pack_bf16x2(__fmul_rn(__fmul_rn(f[2 * e], s), g), __fmul_rn(__fmul_rn(f[2 * e + 1], s), g));
+              nvfp4x8_to_bf16(words[j], j < 2 ? sb0 : sb1, g, o);
               const int chunk = half * 4 + j;
               *reinterpret_cast<uint4*>(bb + row * 128 + ((chunk ^ (row & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
           }
-          // the MMA (async proxy) reads what these generic stores wrote
+          // The MMA (async proxy) reads what these generic stores wrote: the
+          // proxy fence, then an arrival released at CTA scope, as the scale
+          // movers do for TMEM.  The stores are performed in this CTA's own
+          // shared memory before its arrival leaves the CTA, and the pair MMA
+          // reads this CTA's half of B from there.  (A cluster-scope release
+          // on every arrival gave bit-identical results at half the speed.)
           fence_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            if (kCG == 2 && !leader)
-              mbar_arrive_cluster_release(peer_smem(smem_u32(&full[stage]), 0));
-            else
-              mbar_arrive(&full[stage]);
-          }
+          if (lane == 0) arrive_leader(&full[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;

@@ -36,6 +36,7 @@ struct GemmParams {
   const float* alpha_scale;   // nullable: if set, the epilogue uses fl(alpha * alpha_scale[0]) instead
   const float* row_scale;     // row-wise FP8: [M] scales of A's rows
   const float* col_scale;     // row-wise FP8: [N] scales of B's rows (output columns)
+  float w_scale;              // W4A16: the weight's per-tensor scale, applied by the transform warps
   const __nv_bfloat16* bias;  // nullable
   unsigned* fault;
   // fused epilogue (only read by the fused kernel)
@@ -100,7 +101,7 @@ GemmConfig gemm_config(int64_t M, int64_t N, int num_sms);
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,
                         cudaStream_t stream, const DeviceInfo& dev, bool row = false);
 // W4A16: bf16 activations [M, K] x NVFP4 weights [N, K] dequantized in shared
-// memory (p.alpha_mul carries the weight's per-tensor scale, p.alpha = 1);
+// memory (p.w_scale is the weight's per-tensor scale; p.alpha = 1);
 // maps: a = bf16 activations (64-element boxes), b = weight codes (32-byte
 // boxes of this CTA's B rows), sfb = weight scales (one atom per k-tile).
 cudaError_t launch_gemm_w4a16(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, cudaStream_t stream,
