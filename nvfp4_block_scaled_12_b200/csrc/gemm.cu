@@ -261,18 +261,28 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
       // issues the entries j with j % kProducers == pid into stage j % S
       const int my_tiles = p.num_tiles > cluster ? (p.num_tiles - cluster + num_clusters - 1) / num_clusters : 0;
       const int64_t total = static_cast<int64_t>(my_tiles) * p.num_kt;
+      // entry j = t_i * num_kt + kt of this CTA group's t_i-th tile; stage,
+      // phase, tile and k-tile advance incrementally (no 64-bit division on
+      // the way to the first loads)
+      int t_i = 0, kt = pid;
+      while (kt >= p.num_kt) {
+        kt -= p.num_kt;
+        ++t_i;
+      }
+      int stage = pid, cur_t = -1, tm = 0, n0 = 0;
+      uint32_t phase = 0;
       int64_t j = pid;
       for (; j < total; j += kProducers) {
-        const int stage = static_cast<int>(j % S);
-        const uint32_t phase = static_cast<uint32_t>((j / S) & 1);
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
           fault = kFaultProducerWait;
           break;
         }
-        const int tile = cluster + static_cast<int>(j / p.num_kt) * num_clusters;
-        const int kt = static_cast<int>(j % p.num_kt);
-        const int tm = tile % p.tiles_m;
-        const int n0 = (tile / p.tiles_m) * kBN;
+        if (t_i != cur_t) {
+          cur_t = t_i;
+          const int tile = cluster + t_i * num_clusters;
+          tm = tile % p.tiles_m;
+          n0 = (tile / p.tiles_m) * kBN;
+        }
         const int row_block = tm * kCG + static_cast<int>(rank);  // this CTA's 128-row block
         if (leader) mbar_arrive_expect_tx(&full[stage], C::kFullTx);
         if (!kRow) mbar_arrive_expect_tx(&sfin[stage], C::kSfaBytes + C::kSfbBytes + C::kCodeBytes);
@@ -298,6 +308,16 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         } else if (!kRow) {
           tma_load_3d(smem + C::kOffSfa + stage * C::kSfaBytes, &tmap_sfa, &sfin[stage], 0, kt * C::kAtoms, row_block);
           tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * C::kAtoms, n0 >> 7);
+        }
+        kt += kProducers;
+        while (kt >= p.num_kt) {
+          kt -= p.num_kt;
+          ++t_i;
+        }
+        stage += kProducers;
+        if (stage >= S) {
+          stage -= S;
+          phase ^= 1u;
         }
       }
       if (fault != 0u) {
