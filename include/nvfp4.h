@@ -452,6 +452,27 @@ nvfp4_status nvfp4_testing_set_grid_wait(uint64_t limit_ns, uint32_t extra_arriv
 nvfp4_status nvfp4_gemm_tile_shape(int64_t M, int64_t N, int32_t num_sms, int32_t* out);
 
 /*
+ * Launch plan of the GEMMs with the plain epilogue -- nvfp4_gemm,
+ * nvfp4_gemm_scaled, nvfp4_gemm_dynamic (w4a16 = 0) and nvfp4_w4a16_gemm
+ * (w4a16 = 1) -- for an M x N x K problem on num_sms SMs (host only):
+ *   out[0..2] = tile shape as nvfp4_gemm_tile_shape reports it,
+ *   out[3]    = K split: tile groups (CTAs or CTA pairs) that share one
+ *               output tile over disjoint ranges of k-tiles (1, 2 or 4).
+ * When the tiles cannot fill the SMs (a few hundred tokens or fewer) and K is
+ * long enough for the split to pay for its own work, up to 4 CTAs of a
+ * thread-block cluster work on one tile, each over its own k-tile range
+ * (k-tiles of 256 elements for NVFP4, 64 for W4A16), and sum their fp32
+ * partial tiles through distributed shared memory in a fixed order before the
+ * epilogue (so results are deterministic; they may differ from the unsplit
+ * sum in the last bits, within the GEMM's tolerance).  The shape is then the
+ * one of 256 x 192 or 256 x 128 (M > 128) that leaves each CTA group the
+ * fewest k-tiles.  The fused, MXFP8 and row-wise FP8 GEMMs never split K.
+ * Errors: EINVAL (null out, sizes out of range).
+ */
+nvfp4_status nvfp4_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t num_sms, int32_t w4a16,
+                             int32_t* out);
+
+/*
  * Rows per tile of the NVFP4 and MXFP8 quantizers for an [M, K] input on a
  * device with num_sms SMs: 256 once every SM gets at least eight 256-row
  * tiles of 64 columns, else 128.  0 for invalid sizes (M or K out of range,

@@ -76,13 +76,15 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_w4a16_gemm.argtypes = [vp, vp, vp, i64, i64, i64, f32, vp, vp, vp]
     lib.nvfp4_check_fault.argtypes = []
     lib.nvfp4_gemm_tile_shape.argtypes = [i64, i64, i32, ctypes.POINTER(ctypes.c_int32)]
+    lib.nvfp4_gemm_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int32)]
     lib.nvfp4_quantize_tile_rows.argtypes = [i64, i64, i32]
     lib.nvfp4_quantize_tile_rows.restype = ctypes.c_int32
     for name in ("nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm", "nvfp4_gemm_quant",
                  "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_quantize_dynamic_noalloc",
                  "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
                  "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_gemm_tile_shape", "nvfp4_gemm_scaled",
-                 "nvfp4_gemm_quant_scaled", "nvfp4_testing_set_grid_wait", "nvfp4_w4a16_gemm"):
+                 "nvfp4_gemm_quant_scaled", "nvfp4_testing_set_grid_wait", "nvfp4_w4a16_gemm",
+                 "nvfp4_gemm_plan"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -209,6 +211,14 @@ def nvfp4_gemm_tile_shape(M: int, N: int, num_sms: int) -> tuple:
     """(CTAs per tile, tile width, accumulator buffers) the GEMMs take for M x N."""
     out = (ctypes.c_int32 * 3)()
     _check(library().nvfp4_gemm_tile_shape(M, N, num_sms, out))
+    return tuple(out)
+
+
+def nvfp4_gemm_plan(M: int, N: int, K: int, num_sms: int, w4a16: int = 0) -> tuple:
+    """(CTAs per tile, tile width, accumulator buffers, K split) the plain-epilogue
+    GEMMs (w4a16 = 0: NVFP4; 1: W4A16) take for M x N x K."""
+    out = (ctypes.c_int32 * 4)()
+    _check(library().nvfp4_gemm_plan(M, N, K, num_sms, w4a16, out))
     return tuple(out)
 
 

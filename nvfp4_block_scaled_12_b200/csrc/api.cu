@@ -198,10 +198,13 @@ bool product_ok(float g_a, float g_b) {
 // and the operand tensor maps.
 // mx: 8-bit operands (one E4M3 byte per element), with E8M0 scales per 32
 // (MXFP8) or, with row, one fp32 scale per row passed as sfa / sfb.
+// y (bf16 [M, N]) non-null: the plain NVFP4 epilogue, which may split K
+// across a cluster (gemm_plan) and then writes y directly from the cluster's
+// reduction.
 nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M,
                          int64_t N, int64_t K, float alpha, const void* bias, GemmParams* p, GemmTensorMaps* maps,
                          GemmConfig* cfg, const DeviceInfo** dev, bool mx = false, bool row = false,
-                         bool fused = false) {
+                         bool fused = false, void* split_y = nullptr) {
   if (!a || !sfa || !b || !sfb) return fail(NVFP4_EINVAL, "null operand pointer");
   nvfp4_status st = check_rows_k("M", M, "K", K);
   if (st != NVFP4_OK) return st;
@@ -214,10 +217,23 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   st = current_device(dev);
   if (st != NVFP4_OK) return st;
 
-  *cfg = gemm_config(M, N, (*dev)->num_sms);
+  // a k-tile is 128 bytes of every operand row: 256 fp4 or 128 fp8 elements
+  const int64_t row_bytes = mx ? K : K / 2;
+  const int num_kt = static_cast<int>((row_bytes + 127) / 128);
+  int k_split = 1;
+  if (split_y != nullptr && !mx && !row && !fused) {
+    const GemmPlan plan = gemm_plan(M, N, num_kt, (*dev)->num_sms);
+    *cfg = plan.c;
+    k_split = plan.k_split;
+  } else {
+    *cfg = gemm_config(M, N, (*dev)->num_sms);
+  }
   const int bn = cfg->tile_n;
   const int cg = cfg->cta_group;
   *p = GemmParams{};
+  p->k_split = k_split;
+  p->y = static_cast<__nv_bfloat16*>(split_y);
+  p->ldy = static_cast<int32_t>(N);
   p->M = static_cast<int32_t>(M);
   p->N = static_cast<int32_t>(N);
   p->K = static_cast<int32_t>(K);
@@ -226,9 +242,7 @@ nvfp4_status gemm_common(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
   const int64_t tiles = static_cast<int64_t>(p->tiles_m) * p->tiles_n;
   if (tiles > INT32_MAX) return fail(NVFP4_EINVAL, "problem too large");
   p->num_tiles = static_cast<int32_t>(tiles);
-  // a k-tile is 128 bytes of every operand row: 256 fp4 or 128 fp8 elements
-  const int64_t row_bytes = mx ? K : K / 2;
-  p->num_kt = static_cast<int32_t>((row_bytes + 127) / 128);
+  p->num_kt = static_cast<int32_t>(num_kt);
   p->kblocks = static_cast<int32_t>(mx ? K / 32 : K / 64);
   p->alpha = alpha;
   p->alpha_mul = 1.0f;
@@ -551,7 +565,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, 
   GemmTensorMaps maps;
   GemmConfig cg;
   const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev);
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, alpha, bias, &p, &maps, &cg, &dev, false, false, false, y);
   if (st != NVFP4_OK) return st;
   st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
   if (st != NVFP4_OK) return st;
@@ -570,7 +584,7 @@ nvfp4_status nvfp4_gemm_scaled(const uint8_t* a, const uint8_t* sfa, const uint8
   GemmTensorMaps maps;
   GemmConfig cg;
   const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev);
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev, false, false, false, y);
   if (st != NVFP4_OK) return st;
   p.alpha_mul = g_a;
   st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
@@ -594,8 +608,12 @@ nvfp4_status nvfp4_w4a16_gemm(const void* x, const uint8_t* w_codes, const uint8
   const DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != NVFP4_OK) return st;
-  const GemmConfig cg = gemm_config(M, N, dev->num_sms);
+  const GemmPlan plan = gemm_plan(M, N, static_cast<int>(K / 64), dev->num_sms);
+  const GemmConfig cg = plan.c;
   GemmParams p{};
+  p.k_split = plan.k_split;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ldy = static_cast<int32_t>(N);
   p.M = static_cast<int32_t>(M);
   p.N = static_cast<int32_t>(N);
   p.K = static_cast<int32_t>(K);
@@ -639,7 +657,7 @@ nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint
   GemmTensorMaps maps;
   GemmConfig cg;
   const DeviceInfo* dev = nullptr;
-  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev);
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev, false, false, false, y);
   if (st != NVFP4_OK) return st;
   p.alpha_scale = g_a;
   st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
@@ -703,6 +721,20 @@ nvfp4_status nvfp4_gemm_tile_shape(int64_t M, int64_t N, int32_t num_sms, int32_
   out[0] = c.cta_group;
   out[1] = c.tile_n;
   out[2] = c.acc_bufs;
+  return ok();
+}
+
+nvfp4_status nvfp4_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t num_sms, int32_t w4a16, int32_t* out) {
+  if (!out) return fail(NVFP4_EINVAL, "null output pointer");
+  if (M < 1 || M > kMaxDim || N < 8 || N > kMaxDim || K < 64 || K % 64 != 0 || K > kMaxDim || num_sms < 2)
+    return fail(NVFP4_EINVAL, "M=%lld, N=%lld, K=%lld, num_sms=%d out of range", (long long)M, (long long)N,
+                (long long)K, num_sms);
+  const int num_kt = static_cast<int>(w4a16 ? K / 64 : (K / 2 + 127) / 128);
+  const GemmPlan plan = gemm_plan(M, N, num_kt, num_sms);
+  out[0] = plan.c.cta_group;
+  out[1] = plan.c.tile_n;
+  out[2] = plan.c.acc_bufs;
+  out[3] = plan.k_split;
   return ok();
 }
 

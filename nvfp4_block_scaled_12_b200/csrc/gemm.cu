@@ -139,6 +139,10 @@ struct Cfg {
   static_assert(!kWide || kCG == 2, "wide tiles are CTA pairs");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(!kW16 || (!kMx && !kRow), "W4A16 has bf16 activations and NVFP4 weights");
+  // K split: a CTA's fp32 partial tile, 128 rows of kBN + 4 floats (the pad
+  // spreads the rows over the banks), in the idle stage ring
+  static constexpr uint32_t kPartStride = (kBN + 4) * 4;
+  static_assert(kWide || 128 * kPartStride <= kOffEpi, "the partial tile fits the stage ring");
   static_assert(kCodeBytes % 128 == 0 && kSfbBytes % 128 == 0, "TMA destinations stay 128-byte aligned");
 };
 
@@ -193,8 +197,17 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = kCG == 2 ? cluster_ctarank() : 0u;
+  // A cluster is one tile group of kCG CTAs, or, with a K split, p.k_split
+  // such groups that share one output tile over disjoint k-tile ranges; a CTA
+  // pair is cluster ranks 2i, 2i + 1.
+  const uint32_t crank = (kCG == 2 || p.k_split > 1) ? cluster_ctarank() : 0u;
+  const uint32_t rank = crank % kCG;          // CTA within its tile group
+  const uint32_t lead_rank = crank - rank;    // cluster rank of the group leader
   const bool leader = rank == 0;
+  const int split = static_cast<int>(crank) / kCG;  // this group's k-tile range
+  const int kt_begin = static_cast<int>(static_cast<int64_t>(p.num_kt) * split / p.k_split);
+  const int kt_end = static_cast<int>(static_cast<int64_t>(p.num_kt) * (split + 1) / p.k_split);
+  const int my_kt = kt_end - kt_begin;
   // Warp roles.  Standard layout (11 warps): 0 and 10 TMA producers, 1 MMA,
   // 2-5 epilogue, 6-9 scale movers.  Wide layout (16 warps, four warpgroups):
   // 0 and 2 producers, 1 MMA, 3 idle, 4-11 epilogue (two per TMEM lane
@@ -202,8 +215,8 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
   const bool is_producer = C::kWide ? (warp == 0 || warp == 2) : (warp == 0 || warp == 10);
   const bool is_mover = C::kWide ? warp >= 12 : (warp >= 6 && warp <= 9);
   const bool is_epilogue = C::kWide ? (warp >= 4 && warp < 12) : (warp >= 2 && warp <= 5);
-  const int cluster = blockIdx.x / kCG;
-  const int num_clusters = gridDim.x / kCG;
+  const int cluster = blockIdx.x / (kCG * p.k_split);
+  const int num_clusters = gridDim.x / (kCG * p.k_split);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -233,7 +246,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
   }
   tc_fence_before();
   __syncthreads();
-  if (kCG == 2) cluster_sync();  // the peer's barriers are initialised before anyone signals them
+  if (kCG == 2 || p.k_split > 1) cluster_sync();  // the peer's barriers are initialised before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   unsigned fault = 0u;
@@ -241,14 +254,14 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
   // arrive on a barrier that lives in the group leader
   auto arrive_leader = [&](uint64_t* bar) {
     if (kCG == 2 && !leader)
-      mbar_arrive_cluster(peer_smem(smem_u32(bar), 0));
+      mbar_arrive_cluster(peer_smem(smem_u32(bar), lead_rank));
     else
       mbar_arrive(bar);
   };
   // commit to a barrier in every CTA of the group
   auto commit_group = [&](uint64_t* bar) {
     if (kCG == 2)
-      tc_commit_pair(bar, 0x3);
+      tc_commit_pair(bar, static_cast<uint16_t>(0x3u << lead_rank));
     else
       tc_commit(bar);
   };
@@ -260,13 +273,13 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
       // flattened (tile, k-tile) sequence of this CTA group; producer pid
       // issues the entries j with j % kProducers == pid into stage j % S
       const int my_tiles = p.num_tiles > cluster ? (p.num_tiles - cluster + num_clusters - 1) / num_clusters : 0;
-      const int64_t total = static_cast<int64_t>(my_tiles) * p.num_kt;
-      // entry j = t_i * num_kt + kt of this CTA group's t_i-th tile; stage,
-      // phase, tile and k-tile advance incrementally (no 64-bit division on
-      // the way to the first loads)
-      int t_i = 0, kt = pid;
-      while (kt >= p.num_kt) {
-        kt -= p.num_kt;
+      const int64_t total = static_cast<int64_t>(my_tiles) * my_kt;
+      // entry j = t_i * my_kt + (kt - kt_begin) of this CTA group's t_i-th
+      // tile; stage, phase, tile and k-tile advance incrementally (no 64-bit
+      // division on the way to the first loads)
+      int t_i = 0, kt = kt_begin + pid;
+      while (kt >= kt_end) {
+        kt -= my_kt;
         ++t_i;
       }
       int stage = pid, cur_t = -1, tm = 0, n0 = 0;
@@ -293,7 +306,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         const int32_t xa = kW16 ? kt * 64 : kt * kBKBytes;
         const int brow = n0 + static_cast<int>(rank) * C::kBNc;  // this CTA's first B row
         if (kCG == 2) {
-          const uint32_t fb = peer_smem(smem_u32(&full[stage]), 0);
+          const uint32_t fb = peer_smem(smem_u32(&full[stage]), lead_rank);
           tma_load_2d_pair(sa, &tmap_a, fb, xa, row_block * 128);
           if (!kW16) tma_load_2d_pair(sb, &tmap_b, fb, kt * kBKBytes, brow);
         } else {
@@ -310,8 +323,8 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
           tma_load_3d(smem + C::kOffSfb + stage * C::kSfbBytes, &tmap_sfb, &sfin[stage], 0, kt * C::kAtoms, n0 >> 7);
         }
         kt += kProducers;
-        while (kt >= p.num_kt) {
-          kt -= p.num_kt;
+        while (kt >= kt_end) {
+          kt -= my_kt;
           ++t_i;
         }
         stage += kProducers;
@@ -378,7 +391,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        for (int kt = 0; kt < p.num_kt; ++kt) {
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             fault = kFaultMmaWait;
             break;
@@ -396,13 +409,14 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
           // units, so the next 32-byte k-block is +2).
           const uint64_t ad = sdesc_kmajor_sw128(sa), bd = sdesc_kmajor_sw128(sb);
           if (nkb == 4) {
-            const uint32_t first = kt != 0 ? 1u : 0u;
+            const uint32_t first = kt != kt_begin ? 1u : 0u;  // the range's first k-tile starts the sum
             mma(d_tmem, ad, bd, sfa, sfb, 0, first);
             mma(d_tmem, ad + 2, bd + 2, sfa, sfb, 1, 1u);
             mma(d_tmem, ad + 4, bd + 4, sfa, sfb, 2, 1u);
             mma(d_tmem, ad + 6, bd + 6, sfa, sfb, 3, 1u);
           } else {
-            for (int kb = 0; kb < nkb; ++kb) mma(d_tmem, ad + 2 * kb, bd + 2 * kb, sfa, sfb, kb, (kt | kb) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < nkb; ++kb)
+              mma(d_tmem, ad + 2 * kb, bd + 2 * kb, sfa, sfb, kb, (kt != kt_begin || kb != 0) ? 1u : 0u);
           }
           // frees the smem stage and the scale slot once these MMAs have read them
           commit_group(&empty[stage]);
@@ -442,7 +456,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
     for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
       // a 192-wide tile that starts at row 64 of a 128-row scale block
       const bool mid = ((tile / p.tiles_m) * kBN & 127) != 0;
-      for (int kt = 0; kt < p.num_kt; ++kt, ++j) {
+      for (int kt = kt_begin; kt < kt_end; ++kt, ++j) {
         const bool landed = mbar_wait(&sfin[stage], phase, abort_flag);
         __syncwarp();
         if (!__all_sync(0xffffffffu, landed)) {
@@ -567,7 +581,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
       for (int tile = cluster; tile < p.num_tiles && fault == 0u; tile += num_clusters) {
         const int n0 = (tile / p.tiles_m) * kBN;
         const int brow = n0 + static_cast<int>(rank) * C::kBNc;
-        for (int kt = 0; kt < p.num_kt; ++kt) {
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
           const bool landed = mbar_wait(&sfin[stage], phase, abort_flag);
           __syncwarp();
           if (!__all_sync(0xffffffffu, landed)) {
@@ -781,6 +795,24 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
       const int row_base = (tm * kCG + static_cast<int>(rank)) * 128 + q * 32;
       const int row = row_base + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
+      if constexpr (!kFused && !kMx) {
+        if (p.k_split > 1) {
+          // K split: this group's raw partial sums to this CTA's shared memory
+          // (the stage ring is idle: one tile per cluster, all of its k-tiles
+          // consumed), summed across the cluster once every role is done
+          uint8_t* prow = smem + (q * 32 + lane) * C::kPartStride;
+#pragma unroll 1
+          for (int c = 0; c < C::kChunks; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              *reinterpret_cast<uint4*>(prow + c * 128 + v * 16) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+          }
+          continue;
+        }
+      }
       uint32_t sf_word = 0u;
 #pragma unroll 1
       for (int c = 0; c < C::kChunks; ++c) {
@@ -874,10 +906,53 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
       run_epilogue();
   }
 
+  if constexpr (!C::kWide && !kFused && !kMx) {
+    if (p.k_split > 1) {
+      // ------------------------------------------------------------ K-split reduction
+      // Every group's partial tile is in its CTA's shared memory once the
+      // cluster barrier completes.  CTA (split s, pair rank r) then finishes
+      // rows [s * 128 / k_split, (s + 1) * 128 / k_split) of the r-th 128-row
+      // half: the k_split partials summed in split order (so the result is
+      // deterministic), y = bf16(alpha * sum + bias), 16 bytes a thread.
+      tc_fence_before();
+      __syncthreads();
+      cluster_sync();
+      const float alpha = __fmul_rn(p.alpha, p.alpha_scale != nullptr ? *p.alpha_scale : p.alpha_mul);
+      const int rows = 128 / p.k_split;
+      constexpr int kGroupsN = kBN / 8;
+      const int tm = cluster % p.tiles_m;  // one tile per cluster
+      const int n0 = (cluster / p.tiles_m) * kBN;
+      const uint32_t part = smem_u32(smem);
+      for (int it = threadIdx.x; it < rows * kGroupsN; it += C::kThreads) {
+        const int rr = split * rows + it / kGroupsN;
+        const int cg = it % kGroupsN;
+        const int m = (tm * kCG + static_cast<int>(rank)) * 128 + rr;
+        const int n = n0 + cg * 8;
+        if (m >= p.M || n >= p.N) continue;
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int s2 = 0; s2 < p.k_split; ++s2) {
+          const uint32_t src = peer_smem(part + static_cast<uint32_t>(rr) * C::kPartStride + cg * 32,
+                                         static_cast<uint32_t>(s2 * kCG) + rank);
+          const float4 a = ld_shared_cluster_f4(src), b = ld_shared_cluster_f4(src + 16);
+          v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+          v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+        }
+        uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+        if (p.bias != nullptr) bv = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+        const uint4 o = make_uint4(pack_bf16x2(fmaf(alpha, v[0], bf16_lo(bv.x)), fmaf(alpha, v[1], bf16_hi(bv.x))),
+                                   pack_bf16x2(fmaf(alpha, v[2], bf16_lo(bv.y)), fmaf(alpha, v[3], bf16_hi(bv.y))),
+                                   pack_bf16x2(fmaf(alpha, v[4], bf16_lo(bv.z)), fmaf(alpha, v[5], bf16_hi(bv.z))),
+                                   pack_bf16x2(fmaf(alpha, v[6], bf16_lo(bv.w)), fmaf(alpha, v[7], bf16_hi(bv.w))));
+        *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(m) * p.ldy + n) = o;
+      }
+    }
+  }
   if (fault != 0u && lane == 0 && p.fault != nullptr) atomicOr(p.fault, fault);
   tc_fence_before();
   __syncthreads();
-  if (kCG == 2) cluster_sync();  // the peer no longer reads this CTA's smem or signals its barriers
+  // the peers no longer read this CTA's shared memory (the pair MMA, the
+  // K-split reduction) or signal its barriers
+  if (kCG == 2 || p.k_split > 1) cluster_sync();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
@@ -902,6 +977,18 @@ cudaError_t launch(const GemmTensorMaps& m, const GemmParams& p, cudaStream_t st
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = kCG == 2 ? 1 : 0;
+  if (p.k_split > 1) {
+    // K split: one tile per cluster of kCG * k_split CTAs (at most 8, the
+    // portable cluster size); the clusters are independent, so they need not
+    // all be resident at once
+    if (C::kWide || kFused || kMx || kCG * p.k_split > 8) return cudaErrorInvalidConfiguration;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(kCG * p.k_split);
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles * kCG * p.k_split), 1, 1);
+    err = cudaLaunchKernelEx(&cfg, kernel, m.a, m.b, m.sfa, m.sfb, m.y, p);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+  }
   // A persistent grid must be co-resident: as many CTA groups as fit at once,
   // found once per template instance and device (two host threads that race
   // on the first launch compute and store the same value).
@@ -941,6 +1028,48 @@ GemmConfig gemm_config(int64_t M, int64_t N, int num_sms) {
   const int64_t tiles128 = ((M + 255) / 256) * ((N + 127) / 128);
   if (tiles192 < pairs && tiles128 <= pairs) return GemmConfig{2, 128, 2};
   return GemmConfig{2, 192, 2};
+}
+
+GemmPlan gemm_plan(int64_t M, int64_t N, int num_kt, int num_sms) {
+  const GemmConfig base = gemm_config(M, N, num_sms);
+  if (base.cta_group == 2 && base.tile_n == 256) return GemmPlan{base, 1};  // a tile for every CTA pair
+  // Cost of a shape, in k-tiles of one CTA group: the tiles in waves of the
+  // co-resident groups; or, with few tiles, the share of the K range of a
+  // power-of-two split plus kSplitCost for the split's own work (writing the
+  // partial tile, two cluster barriers, the reduction through distributed
+  // shared memory).  A split keeps every cluster within 4 CTAs and all of them
+  // resident at once (at most 7/8 of the SMs: clusters of 4 CTAs with this
+  // kernel's shared memory fit 33 at a time on 148 SMs, of 8 only 15), and at
+  // least one k-tile to a range.
+  constexpr int64_t kSplitCost = 6;
+  auto cost = [&](const GemmConfig& c, int* ks_out) {
+    const int64_t groups = num_sms / c.cta_group;
+    const int64_t tiles = ((M + 128 * c.cta_group - 1) / (128 * c.cta_group)) * ((N + c.tile_n - 1) / c.tile_n);
+    *ks_out = 1;
+    if (tiles > groups) return static_cast<int64_t>(num_kt) * ((tiles + groups - 1) / groups);
+    int64_t best_c = num_kt;
+    for (int ks = 2; ks * c.cta_group <= 4 && ks <= num_kt && tiles * ks * c.cta_group * 8 <= num_sms * 7; ks *= 2) {
+      const int64_t cc = (num_kt + ks - 1) / ks + kSplitCost;
+      if (cc < best_c) {
+        best_c = cc;
+        *ks_out = ks;
+      }
+    }
+    return best_c;
+  };
+  GemmPlan best{base, 1};
+  int64_t best_cost = cost(base, &best.k_split);
+  if (M > 128) {
+    for (const GemmConfig c : {GemmConfig{2, 192, 2}, GemmConfig{2, 128, 2}}) {
+      int ks = 1;
+      const int64_t cc = cost(c, &ks);
+      if (cc < best_cost) {
+        best = GemmPlan{c, ks};
+        best_cost = cc;
+      }
+    }
+  }
+  return best;
 }
 
 cudaError_t launch_gemm_w4a16(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, cudaStream_t stream,

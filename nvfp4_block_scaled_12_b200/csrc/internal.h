@@ -37,6 +37,9 @@ struct GemmParams {
   const float* row_scale;     // row-wise FP8: [M] scales of A's rows
   const float* col_scale;     // row-wise FP8: [N] scales of B's rows (output columns)
   float w_scale;              // W4A16: the weight's per-tensor scale, applied by the transform warps
+  int32_t k_split;            // tile groups per cluster that share one output tile (K split); 1 = none
+  __nv_bfloat16* y;           // K split: the bf16 output [M, ldy], written by the cluster's reduction
+  int32_t ldy;
   const __nv_bfloat16* bias;  // nullable
   unsigned* fault;
   // fused epilogue (only read by the fused kernel)
@@ -96,6 +99,15 @@ struct GemmConfig {
   int acc_bufs;   // accumulator buffers in TMEM
 };
 GemmConfig gemm_config(int64_t M, int64_t N, int num_sms);
+// Tile shape and K split of a GEMM whose epilogue is the plain one (NVFP4 and
+// W4A16 with bias): when the tiles cannot fill the SMs, up to 8 CTAs (4 CTA
+// pairs) of a cluster share one tile over disjoint k-tile ranges.  num_kt:
+// k-tiles of the problem (256 elements for NVFP4, 64 for W4A16).
+struct GemmPlan {
+  GemmConfig c;
+  int k_split;
+};
+GemmPlan gemm_plan(int64_t M, int64_t N, int num_kt, int num_sms);
 // mx: MXFP8 operands (E4M3 codes [rows, K], E8M0 scales) instead of NVFP4.
 // row: row-wise FP8 (8-bit operands without block scales; requires mx).
 cudaError_t launch_gemm(const GemmTensorMaps& m, const GemmParams& p, const GemmConfig& c, bool fused, bool mx,

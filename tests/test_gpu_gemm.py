@@ -256,3 +256,45 @@ def test_wide_tiles_are_deterministic(F):
 
 def test_no_kernel_reported_a_fault(F):
     F.nvfp4_check_fault()
+
+
+def _plan(F, m, n, k, w16=0):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return F.nvfp4_gemm_plan(m, n, k, sms, w16)
+
+
+@pytest.mark.parametrize("m,n,k,ks", [(100, 3072, 3072, 4), (77, 1000, 4160, 4), (16, 3072, 15360, 4),
+                                      (1, 8, 4096, 4), (300, 520, 15360, 2), (129, 392, 4096, 2)])
+def test_split_k_matches_the_oracle(F, m, n, k, ks):
+    # A few hundred tokens or fewer: CTAs of one cluster share each output
+    # tile over disjoint k-tile ranges and sum their partial tiles through
+    # distributed shared memory; ragged M, N and a last k-tile of one k-block.
+    assert _plan(F, m, n, k)[3] == ks
+    _check_linear(F, synth.LinearWorkload(f"split_{m}x{n}x{k}", m, k, n, seed=m + 7 * n + k))
+
+
+def test_split_k_exact_accumulation_is_bit_exact(F):
+    # every partial sum and their sum are exact in fp32, so the split result
+    # equals the rounded exact result bit for bit
+    rng = np.random.default_rng(33)
+    M, N, K = 100, 384, 4096  # |partial sums| < 2^20, a step of 2^-4: exact in fp32
+    assert _plan(F, M, N, K)[3] == 4
+    a_codes = rng.integers(0, 256, (M, K // 2)).astype(np.uint8)
+    b_codes = rng.integers(0, 256, (N, K // 2)).astype(np.uint8)
+    pow2 = np.array([0x30, 0x38, 0x40], np.uint8)
+    a_sf, b_sf = rng.choice(pow2, (M, K // 16)), rng.choice(pow2, (N, K // 16))
+    bias = O.round_to_bf16(rng.integers(-64, 64, N) * 0.5)
+    y = _run_raw(F, a_codes, a_sf, b_codes, b_sf, alpha=0.5, bias=bias.astype(np.float32))
+    want = O.round_to_bf16(O.gemm_ref(a_codes, a_sf, 1.0, b_codes, b_sf, 1.0, None) * 0.5 + bias)
+    bad = np.argwhere(y != want)
+    assert bad.size == 0, f"{bad.shape[0]} differ, first {bad[:4].tolist()}"
+
+
+def test_split_k_is_deterministic(F):
+    wl = synth.LinearWorkload("det_split", 300, 15360, 520, seed=11)
+    assert _plan(F, wl.m, wl.n, wl.k)[3] == 2
+    xq, wq = _gpu_layer(F, wl.activations(), wl.weight())
+    b = wl.bias_vec().cuda()
+    ys = [F.gemm(xq, wq, bias=b) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])

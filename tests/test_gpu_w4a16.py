@@ -55,15 +55,15 @@ def test_dequantize_the_weights_the_quantizer_wrote(F):
     assert_bytes_equal(_bf16_bytes(got), _bf16_bytes(want), "weights")
 
 
-def _shape(F, m, n):
+def _plan(F, m, n, k):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    return F.nvfp4_gemm_tile_shape(m, n, sms)
+    return F.nvfp4_gemm_plan(m, n, k, sms, 1)
 
 
 def _w4a16_check(F, wl, rows=None, cols=None, shape=None):
     x, w, bias = wl.activations(), wl.weight(), wl.bias_vec()
     if shape is not None:
-        assert _shape(F, wl.m, wl.n) == shape
+        assert _plan(F, wl.m, wl.n, wl.k) == shape
     g = float(O.global_scale(O.tensor_amax(f32(w))))
     wq = F.quantize(w.cuda(), g)
     y = F.linear_w4a16(x.cuda(), wq, None if bias is None else bias.cuda())
@@ -91,9 +91,9 @@ def test_w4a16_linear_matches_the_oracle(F, m):
     _w4a16_check(F, synth.LinearWorkload(f"w4a16_m{m}", m, 3072, 768, seed=70 + m))
 
 
-@pytest.mark.parametrize("m,n,k,shape", [(1, 8, 64, (1, 192, 2)), (77, 1000, 4160, (1, 192, 2)),
-                                         (300, 520, 1088, (2, 128, 2)), (1000, 2880, 3136, (2, 192, 2)),
-                                         (2341, 2056, 1024, (2, 256, 1))])
+@pytest.mark.parametrize("m,n,k,shape", [(1, 8, 64, (1, 192, 2, 1)), (77, 1000, 4160, (1, 192, 2, 4)),
+                                         (300, 520, 1088, (2, 128, 2, 2)), (1000, 2880, 3136, (2, 192, 2, 1)),
+                                         (2341, 2056, 1024, (2, 256, 1, 1)), (512, 3072, 3072, (2, 192, 2, 2))])
 def test_w4a16_every_tile_shape_ragged(F, m, n, k, shape):
     wl = synth.LinearWorkload(f"w4a16_{m}x{n}x{k}", m, k, n, seed=m + n + k)
     rng = np.random.default_rng(m + n)
@@ -105,7 +105,7 @@ def test_w4a16_mlp_up_sampled(F):
     # the MLP-up shape, M = 4608 (wide tiles): all columns of sampled rows
     wl = synth.MLP_UP
     rows = np.sort(np.random.default_rng(5).choice(wl.m, 48, replace=False))
-    _w4a16_check(F, wl, rows=rows, shape=(2, 256, 1))
+    _w4a16_check(F, wl, rows=rows, shape=(2, 256, 1, 1))
 
 
 @pytest.mark.parametrize("m,n", [(100, 384), (512, 768), (1000, 2880), (2304, 2304)])
@@ -128,6 +128,16 @@ def test_w4a16_exact_accumulation_is_bit_exact(F, m, n):
     got = y.float().cpu().numpy()
     bad = np.argwhere(got != want)
     assert bad.size == 0, f"{bad.shape[0]} differ, first {bad[:4].tolist()}"
+
+
+def test_w4a16_split_k_is_deterministic(F):
+    wl = synth.LinearWorkload("w4a16_det_split", 100, 3072, 3072, seed=12)
+    assert _plan(F, wl.m, wl.n, wl.k)[3] == 4
+    x, w = wl.activations().cuda(), wl.weight().cuda()
+    wq = F.quantize(w, F.global_scale(w))
+    ys = [F.linear_w4a16(x, wq) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
 
 
 @pytest.mark.parametrize("m,n,row,kblk", [(100, 384, 37, 3), (100, 384, 200, 15), (512, 768, 130, 9),

@@ -65,3 +65,34 @@ def test_quantize_tile_rows_is_zero_for_invalid_sizes():
     assert F.nvfp4_quantize_tile_rows(0, 64, SMS) == 0
     assert F.nvfp4_quantize_tile_rows(4, 96, SMS) == 0
     assert F.nvfp4_quantize_tile_rows(4, 64, 0) == 0
+
+
+@pytest.mark.parametrize("m,n,k,w16,want,why", [
+    (100, 3072, 3072, 0, (1, 192, 2, 4), "16 tiles of 128 x 192: four CTAs share each tile, 12 k-tiles -> 3 each"),
+    (100, 3072, 3072, 1, (1, 192, 2, 4), "W4A16: 48 k-tiles of 64 -> 12 a CTA"),
+    (512, 3072, 3072, 0, (2, 128, 2, 1), "12 k-tiles: a split would save less than its own work"),
+    (512, 3072, 3072, 1, (2, 192, 2, 2), "W4A16, 48 k-tiles: 32 pair tiles of 192 split in two"),
+    (1024, 3072, 3072, 0, (2, 192, 2, 1), "64 pair tiles already fill the pairs"),
+    (4608, 12288, 3072, 0, (2, 256, 1, 1), "wide tiles never split"),
+    (128, 256, 256, 0, (1, 192, 2, 1), "one k-tile: nothing to split"),
+    (300, 520, 1088, 1, (2, 128, 2, 2), "two CTA pairs (4 CTAs) to a cluster at most"),
+    (16, 3072, 15360, 0, (1, 192, 2, 4), "4 CTAs to a cluster at most"),
+    (300, 520, 15360, 0, (2, 128, 2, 2), "a long K splits over CTA pairs too"),
+])
+def test_gemm_plan_table(m, n, k, w16, want, why):
+    assert F.nvfp4_gemm_plan(m, n, k, SMS, w16) == want, why
+
+
+def test_gemm_plan_keeps_every_cluster_within_4_ctas_resident_at_once():
+    for m in (1, 37, 128, 129, 300, 512, 777, 1024, 2000):
+        for n in (8, 192, 1000, 3072, 12288):
+            for k in (64, 256, 320, 3072, 15360):
+                for w16 in (0, 1):
+                    cg, bn, acc, ks = F.nvfp4_gemm_plan(m, n, k, SMS, w16)
+                    num_kt = k // 64 if w16 else (k // 2 + 127) // 128
+                    assert ks in (1, 2, 4) and cg * ks <= 4 and ks <= num_kt
+                    tiles = ((m + 128 * cg - 1) // (128 * cg)) * ((n + bn - 1) // bn)
+                    assert ks == 1 or tiles * ks * cg * 8 <= SMS * 7  # every split cluster resident at once
+                    if ks > 1:
+                        assert (cg, bn) != (2, 256)  # the wide tiles never split
+                        assert (num_kt + ks - 1) // ks + 6 < num_kt  # the split saves more than it costs
