@@ -634,7 +634,11 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
   // chunks are quantized (two 16-element blocks) into the next layer's codes
   // and swizzled scales (sf_word collects the 64-column group's scale word).
   const int m_padded = (p.M + 127) & ~127;  // rows of the next layer's scale buffer
-  auto emit_chunk = [&](uint32_t (&w)[16], int n, int row_base, uint8_t* stage_buf, int& buf, uint32_t& sf_word) {
+  // (pend holds the codes of a 64-column group's first chunk until its second
+  // one completes the row's 32 bytes, written as one whole sector)
+  const bool codes32 = (reinterpret_cast<uintptr_t>(p.codes_next) & 31u) == 0;
+  auto emit_chunk = [&](uint32_t (&w)[16], int n, int row_base, uint8_t* stage_buf, int& buf, uint32_t& sf_word,
+                        uint32_t (&pend)[4]) {
     const int row = row_base + lane;
     int act = NVFP4_ACT_NONE, dst = NVFP4_DST_BF16, out_col = n;
     if (kFused) {
@@ -674,10 +678,22 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         blk[2 * j + 1] = bf16_hi(w[8 + j]);
       }
       const uint32_t s1 = quantize_block16(blk, g, d6, c2, c3);
-      if (row < p.M)
-        *reinterpret_cast<uint4*>(p.codes_next + static_cast<size_t>(row) * (p.k_next >> 1) + (out_col >> 1)) =
-            make_uint4(c0, c1, c2, c3);
       const int csf = out_col >> 4;  // scale column of the first block (even)
+      uint8_t* crow = p.codes_next + static_cast<size_t>(row) * (p.k_next >> 1) + (out_col >> 1);
+      if ((csf & 3) == 0) {
+        pend[0] = c0;
+        pend[1] = c1;
+        pend[2] = c2;
+        pend[3] = c3;
+      } else if (row < p.M) {  // the row's 32 bytes of this 64-column group
+        if (codes32) {
+          const uint32_t cw[8] = {pend[0], pend[1], pend[2], pend[3], c0, c1, c2, c3};
+          st_global_v8(crow - 16, cw);
+        } else {
+          *reinterpret_cast<uint4*>(crow - 16) = make_uint4(pend[0], pend[1], pend[2], pend[3]);
+          *reinterpret_cast<uint4*>(crow) = make_uint4(c0, c1, c2, c3);
+        }
+      }
       sf_word |= (s0 | (s1 << 8)) << (8 * (csf & 3));
       if ((csf & 3) == 2) {  // the 64-column group is complete
         const uint32_t word = row < p.M ? sf_word : 0u;  // padding rows of the scale buffer are zero
@@ -738,6 +754,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
       const int row = row_base + lane;
       const float sa = kRow ? (row < p.M ? __ldg(p.row_scale + row) : 0.0f) : 0.0f;
       uint32_t sf_word = 0u;
+      uint32_t pend[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int n = c0 + c * 32;
@@ -764,7 +781,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
                                        fmaf(a1, __uint_as_float(r[j + 1]), bf16_hi(bw[t])));
           }
         }
-        emit_chunk(w, n, row_base, stage_buf, buf, sf_word);
+        emit_chunk(w, n, row_base, stage_buf, buf, sf_word, pend);
       }
     }
     if (lane == 0) bulk_wait<0>();
@@ -814,6 +831,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         }
       }
       uint32_t sf_word = 0u;
+      uint32_t pend[4] = {0u, 0u, 0u, 0u};
 #pragma unroll 1
       for (int c = 0; c < C::kChunks; ++c) {
         uint32_t r[32];
@@ -859,7 +877,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
                                          fmaf(alpha, __uint_as_float(r[8 * g + 2 * t + 1]), bf16_hi(bw[t])));
           }
         }
-        emit_chunk(w, n, row_base, stage_buf, buf, sf_word);
+        emit_chunk(w, n, row_base, stage_buf, buf, sf_word, pend);
       }
       if (++acc == kAcc) {
         acc = 0;
