@@ -254,10 +254,6 @@ def test_wide_tiles_are_deterministic(F):
     assert torch.equal(y1, y2)
 
 
-def test_no_kernel_reported_a_fault(F):
-    F.nvfp4_check_fault()
-
-
 def _plan(F, m, n, k, w16=0):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     return F.nvfp4_gemm_plan(m, n, k, sms, w16)
@@ -298,3 +294,15 @@ def test_split_k_is_deterministic(F):
     ys = [F.gemm(xq, wq, bias=b) for _ in range(3)]
     torch.cuda.synchronize()
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+
+
+def test_long_k(F):
+    # K = 65536: 256 k-tiles, split over CTA pairs, offsets far past the
+    # sizes of the other tests
+    wl = synth.LinearWorkload("long_k", 300, 65536, 256, seed=99)
+    assert _plan(F, wl.m, wl.n, wl.k)[3] > 1
+    _check_linear(F, wl)
+
+
+def test_no_kernel_reported_a_fault(F):
+    F.nvfp4_check_fault()
