@@ -579,7 +579,9 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
     // 128-byte-swizzled K-major layout the MMA descriptors describe:
     //   w = bf16_rn(fl(fl(e2m1(q) * e4m3(s)) * g))   (the first product exact)
     // Work item i of the 2 * kBNc per k-tile = half i % 2 (32 elements, two
-    // 16-element blocks) of row i / 2; the four warps take every 128th item.
+    // 16-element blocks) of row i / 2; the four warps take every 128th item,
+    // two at a time (one transform warp per scheduler: the second item's
+    // independent chain hides the first one's latencies).
     if constexpr (kW16) {
       const int t = (warp & 3) * 32 + lane;
       const float g = p.w_scale;  // the weight's per-tensor scale
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
           const uint8_t* cb = smem + C::kOffCode + stage * C::kCodeBytes;
           const uint8_t* sb = smem + C::kOffSfb + stage * C::kSfbBytes;
           uint8_t* bb = smem + C::kOffB + stage * C::kBBytes;
-#pragma unroll 1
+#pragma unroll 2
           for (int i = t; i < 2 * C::kBNc; i += 128) {
             const int row = i >> 1, half = i & 1;
             const int rg = brow + row;  // B row in the weight (rows past N arrived zero-filled)
