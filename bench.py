@@ -590,6 +590,25 @@ def run_ours(args):
         F.gemm(xq_dyn, wq, bias=bias, y=y, stream=stream)
 
     ld_ms = median_ms(linear_dynamic)
+    # the one-pass dynamic scale: the amax of a layer's input emitted by the
+    # previous layer's GEMM epilogue (timed here on the MLP-up GEMM itself),
+    # then the quantize that derives g from it on the device
+    amax_x = torch.empty(1, dtype=torch.float32, device=device)
+    amax_xl = torch.empty(1, dtype=torch.float32, device=device)
+    amax_x.fill_(float(x.float().abs().max()))
+    amax_xl.fill_(float(xl.float().abs().max()))
+    xq_fa = F.quantize_from_amax(x, amax_x, stream=stream)
+    xlq_fa = F.quantize_from_amax(xl, amax_xl, stream=stream)
+    qa_ms = median_ms(lambda: F.quantize_from_amax(x, amax_x, out=xq_fa, stream=stream))
+    qal_ms = median_ms(lambda: F.quantize_from_amax(xl, amax_xl, out=xlq_fa, stream=stream))
+    amax_y = torch.zeros(1, dtype=torch.float32, device=device)
+    ga_ms = median_ms(lambda: F.gemm(xq, wq, bias=bias, y=y, amax_out=amax_y, stream=stream))
+
+    def linear_from_amax():
+        F.quantize_from_amax(x, amax_x, out=xq_fa, stream=stream)
+        F.gemm(xq_fa, wq, bias=bias, y=y, stream=stream)
+
+    lfa_ms = median_ms(linear_from_amax)
     F.nvfp4_check_fault()
     # the MXFP8 variant on the same MLP-up shape: E4M3 activations and
     # weights with one E8M0 scale per 32 elements, no per-tensor scale
@@ -666,6 +685,15 @@ def run_ours(args):
                 "linear_dynamic": {
                     "ms": ld_ms, "tflops": flops / (ld_ms * 1e-3) / 1e12,
                     "note": "MLP-up step with the measured scale: quantize_dynamic + GEMM reading g on the device"},
+                "quantize_from_amax": {
+                    "ms": qa_ms, "gbs": M * K * QUANT_BYTES_PER_ELEM / (qa_ms * 1e-3) / 1e9,
+                    "frac_of_hbm": M * K * QUANT_BYTES_PER_ELEM / (qa_ms * 1e-3) / 1e9 / hbm,
+                    "ms_4608x12288": qal_ms,
+                    "frac_of_hbm_4608x12288": xl.numel() * QUANT_BYTES_PER_ELEM / (qal_ms * 1e-3) / 1e9 / hbm,
+                    "gemm_with_amax_ms": ga_ms, "linear_ms": lfa_ms,
+                    "note": "one-pass dynamic scale: g derived on the device from an amax the previous layer's "
+                            "GEMM epilogue emitted (gemm_with_amax_ms: the MLP-up GEMM measuring max|Y| of its "
+                            "own output); linear = that quantize + the GEMM reading g on the device"},
                 "mxfp8": {
                     "quantize_ms": q8_ms,
                     "quantize_gbs": M * K * MX_QUANT_BYTES_PER_ELEM / (q8_ms * 1e-3) / 1e9,

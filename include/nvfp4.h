@@ -152,7 +152,27 @@ nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K,
                                     void* workspace, size_t workspace_bytes,
                                     void* stream);
 
-/* Bytes of device scratch nvfp4_quantize_dynamic_noalloc holds per device. */
+/*
+ * The dynamic-scale quantize in one pass, for an activation whose amax was
+ * measured already (by nvfp4_gemm_amax when the previous layer produced it):
+ *     g = 0                                   if amax[0] == 0
+ *         min(max(fl(amax[0] / 2688), 2^-64), 2^64)  otherwise
+ *     codes, sf = nvfp4_quantize(x, g)   (all zero when g == 0)
+ * -- the rule of nvfp4_quantize_dynamic, with the amax given instead of
+ * measured.  The kernel reads amax on the device (work earlier on `stream`
+ * may write it); nothing is read back to the host.
+ *   x, M, K, codes, sf  as nvfp4_quantize.
+ *   amax       device pointer to one non-negative float (4-byte aligned).
+ *   scale_out  2 device floats (4-byte aligned), written: [0] = amax,
+ *              [1] = g (pass &scale_out[1] to nvfp4_gemm_dynamic).
+ * One launch of the static quantizer's grid; no workspace.
+ * Errors: EINVAL (sizes, null), EALIGN, EARCH, ECUDA.
+ */
+nvfp4_status nvfp4_quantize_from_amax(const void* x, int64_t M, int64_t K, const float* amax,
+                                      uint8_t* codes, uint8_t* sf, float* scale_out,
+                                      void* stream);
+
+/* Bytes of device scratch nvfp4_quantize_dynamic_noalloc holds per device. *//* Bytes of device scratch nvfp4_quantize_dynamic_noalloc holds per device. */
 #define NVFP4_NOALLOC_SCRATCH_BYTES 256
 
 /*
@@ -239,7 +259,32 @@ nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint
                                 float g_b, const float* g_a, const void* bias, void* y,
                                 void* stream);
 
-/* One column range of the fused epilogue. */
+/*
+ * The GEMM of nvfp4_gemm_scaled / nvfp4_gemm_dynamic that also measures its
+ * output for the next layer's dynamic scale (the survey's "amax emitted by the
+ * previous layer's epilogue": the next layer then quantizes in one pass with
+ * nvfp4_quantize_from_amax instead of the two passes of
+ * nvfp4_quantize_dynamic).
+ *     Y = bf16( fl(g * g_b) * acc + bias ),  g = g_a_device ? g_a_device[0] : g_a
+ *     amax_out[0] = max(amax_out[0], max |Y[m, n]|)  over the M x N outputs
+ * The maximum is taken over the bf16 values written (a NaN counts as +inf)
+ * and folded in with an atomic max on the float's bit pattern, so amax_out[0]
+ * must hold a non-negative float on entry (zero it to measure one GEMM; leave
+ * it to take the maximum over several).
+ *   g_a         the activation's per-tensor scale (used when g_a_device is
+ *               NULL; then g_a * g_b must be finite)
+ *   g_a_device  nullable device pointer to one float (4-byte aligned), e.g.
+ *               &scale_out[1] of a dynamic or one-pass quantize
+ *   g_b         the weight's per-tensor scale, finite
+ *   amax_out    device pointer to one float (4-byte aligned)
+ * Other arguments and errors as nvfp4_gemm.
+ */
+nvfp4_status nvfp4_gemm_amax(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                             const uint8_t* sfb, int64_t M, int64_t N, int64_t K,
+                             float g_a, const float* g_a_device, float g_b,
+                             const void* bias, void* y, float* amax_out, void* stream);
+
+/* One column range of the fused epilogue. *//* One column range of the fused epilogue. */
 typedef struct nvfp4_colrange {
   int64_t begin;   /* first GEMM output column of the range              */
   int64_t end;     /* one past the last column                           */

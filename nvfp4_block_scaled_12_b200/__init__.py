@@ -62,6 +62,8 @@ def _load() -> ctypes.CDLL:
     lib.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.nvfp4_gemm_dynamic.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, vp, vp, vp]
     lib.nvfp4_gemm_scaled.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, f32, vp, vp, vp]
+    lib.nvfp4_gemm_amax.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, vp, f32, vp, vp, vp, vp]
+    lib.nvfp4_quantize_from_amax.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
     lib.nvfp4_gemm_quant_scaled.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, f32, vp, ctypes.POINTER(ColRange),
                                             i32, vp, i64, f32, vp, vp, i64, vp]
     lib.nvfp4_testing_set_grid_wait.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
@@ -84,7 +86,7 @@ def _load() -> ctypes.CDLL:
                  "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
                  "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_gemm_tile_shape", "nvfp4_gemm_scaled",
                  "nvfp4_gemm_quant_scaled", "nvfp4_testing_set_grid_wait", "nvfp4_w4a16_gemm",
-                 "nvfp4_gemm_plan"):
+                 "nvfp4_gemm_plan", "nvfp4_gemm_amax", "nvfp4_quantize_from_amax"):
         getattr(lib, name).restype = ctypes.c_int
     lib.nvfp4_last_error.argtypes = []
     lib.nvfp4_last_error.restype = ctypes.c_char_p
@@ -132,6 +134,11 @@ def nvfp4_quantize_dynamic_noalloc(x: int, M: int, K: int, codes: int, sf: int, 
     _check(library().nvfp4_quantize_dynamic_noalloc(x, M, K, codes, sf, scale_out, stream))
 
 
+def nvfp4_quantize_from_amax(x: int, M: int, K: int, amax: int, codes: int, sf: int, scale_out: int,
+                             stream: int) -> None:
+    _check(library().nvfp4_quantize_from_amax(x, M, K, amax, codes, sf, scale_out, stream))
+
+
 def nvfp4_swizzle_sf(sf_linear: int, rows: int, k: int, sf_swizzled: int, stream: int) -> None:
     _check(library().nvfp4_swizzle_sf(sf_linear, rows, k, sf_swizzled, stream))
 
@@ -144,6 +151,12 @@ def nvfp4_gemm(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, alpha
 def nvfp4_gemm_scaled(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_a: float, g_b: float,
                       bias: int, y: int, stream: int) -> None:
     _check(library().nvfp4_gemm_scaled(a, sfa, b, sfb, M, N, K, g_a, g_b, bias or None, y, stream))
+
+
+def nvfp4_gemm_amax(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_a: float, g_a_device: int,
+                    g_b: float, bias: int, y: int, amax_out: int, stream: int) -> None:
+    _check(library().nvfp4_gemm_amax(a, sfa, b, sfb, M, N, K, g_a, g_a_device or None, g_b, bias or None, y,
+                                     amax_out, stream))
 
 
 def nvfp4_gemm_dynamic(a: int, sfa: int, b: int, sfb: int, M: int, N: int, K: int, g_b: float, g_a: int,
@@ -360,6 +373,33 @@ def quantize_dynamic(x, out: Optional[NVFP4Tensor] = None, workspace=None, strea
     return out
 
 
+def quantize_from_amax(x, amax, out: Optional[NVFP4Tensor] = None, stream=None) -> NVFP4Tensor:
+    """Quantize bf16 ``x`` [M, K] in one pass with the dynamic rule's scale
+    derived on the device from ``amax`` (a float32 device tensor whose first
+    element is max|x|, e.g. the ``amax_out`` of the GEMM that produced x).  The
+    result's ``scale`` holds [amax, g] on the device, as for quantize_dynamic."""
+    torch = _torch()
+    dev = torch.cuda.current_device()
+    M, K = x.shape
+    _need(x, torch.bfloat16, None, "x", dev=dev)
+    _need(amax, torch.float32, None, "amax", dev=dev)
+    if out is None:
+        out = NVFP4Tensor(torch.empty(M, K // 2, dtype=torch.uint8, device=x.device),
+                          torch.empty(nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=x.device), None, M, K)
+    else:
+        _need(out.codes, torch.uint8, None, "out.codes", M * K // 2, dev=dev)
+        _need(out.sf, torch.uint8, None, "out.sf", nvfp4_sf_bytes(M, K), dev=dev)
+        if (out.rows, out.k) != (M, K):
+            raise ValueError(f"out is [{out.rows}, {out.k}], x is [{M}, {K}]")
+    if out.scale is None:
+        out.scale = torch.empty(2, dtype=torch.float32, device=x.device)
+    _need(out.scale, torch.float32, None, "out.scale", 2, dev=dev)
+    nvfp4_quantize_from_amax(_ptr(x), M, K, _ptr(amax), _ptr(out.codes), _ptr(out.sf), _ptr(out.scale),
+                             _stream(stream))
+    out.g = None
+    return out
+
+
 @dataclass
 class MXFP8Tensor:
     """A [rows, k] MXFP8 tensor on the GPU: E4M3 codes (one byte per element)
@@ -515,10 +555,13 @@ def swizzle_sf(sf_linear, rows: int, k: int, stream=None):
     return out
 
 
-def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = None, y=None, stream=None):
+def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = None, y=None, stream=None,
+         amax_out=None):
     """y = bf16(alpha * a_hat @ b_hat^T + bias).  Without ``alpha`` the
     library forms alpha = fl32(g_a * g_b) from the two per-tensor scales (the
-    activation's read on the device when it was measured there)."""
+    activation's read on the device when it was measured there).  With
+    ``amax_out`` (a float32 device tensor) the epilogue also folds max|y|
+    into amax_out[0] (an atomic max: zero it first to measure this y)."""
     torch = _torch()
     dev = torch.cuda.current_device()
     if a.k != b.k:
@@ -533,7 +576,14 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, bias=None, alpha: Optional[float] = Non
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a.codes.device)
     _need(y, torch.bfloat16, (M, N), "y", dev=dev)
-    if alpha is not None:
+    if amax_out is not None:
+        _need(amax_out, torch.float32, None, "amax_out", dev=dev)
+        # alpha whole (times 1), or the two scales, the activation's possibly on the device
+        g_a, g_a_dev, g_b = ((float(alpha), 0, 1.0) if alpha is not None else
+                             (0.0, _ptr(a.scale) + 4, float(b.g)) if a.g is None else (float(a.g), 0, float(b.g)))
+        nvfp4_gemm_amax(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, g_a, g_a_dev, g_b,
+                        _ptr(bias), _ptr(y), _ptr(amax_out), _stream(stream))
+    elif alpha is not None:
         nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(b.codes), _ptr(b.sf), M, N, K, float(alpha), _ptr(bias),
                    _ptr(y), _stream(stream))
     elif a.g is None:

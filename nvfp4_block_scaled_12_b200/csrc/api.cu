@@ -487,6 +487,28 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
   return ok();
 }
 
+nvfp4_status nvfp4_quantize_from_amax(const void* x, int64_t M, int64_t K, const float* amax, uint8_t* codes,
+                                      uint8_t* sf, float* scale_out, void* stream) {
+  if (!x || !amax || !codes || !sf || !scale_out) return fail(NVFP4_EINVAL, "null pointer");
+  if (check_rows_k("M", M, "K", K) != NVFP4_OK) return NVFP4_EINVAL;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf))
+    return fail(NVFP4_EALIGN, "x, codes and sf must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(amax) & 3u) != 0 || (reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0)
+    return fail(NVFP4_EALIGN, "amax and scale_out must be 4-byte aligned");
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = current_device(&dev);
+  if (st != NVFP4_OK) return st;
+  CUtensorMap tx;
+  const int tile_rows = quantize_tile_rows(M, K, dev->num_sms);
+  st = make_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, K * 2, 64, static_cast<uint32_t>(tile_rows),
+                 CU_TENSOR_MAP_SWIZZLE_128B, "x");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_quantize_from_amax(tx, tile_rows, M, K, amax, codes, sf, scale_out,
+                                            static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
+}
+
 nvfp4_status nvfp4_quantize_dynamic(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
                                     float* scale_out, void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !codes || !sf || !scale_out || !workspace) return fail(NVFP4_EINVAL, "null pointer");
@@ -667,6 +689,32 @@ nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint
   return ok();
 }
 
+
+nvfp4_status nvfp4_gemm_amax(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
+                             int64_t M, int64_t N, int64_t K, float g_a, const float* g_a_device, float g_b,
+                             const void* bias, void* y, float* amax_out, void* stream) {
+  if (!y || !amax_out) return fail(NVFP4_EINVAL, "null output pointer");
+  if (!aligned16(y)) return fail(NVFP4_EALIGN, "y must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(amax_out) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(g_a_device) & 3u) != 0)
+    return fail(NVFP4_EALIGN, "amax_out and g_a_device must be 4-byte aligned");
+  if (g_a_device == nullptr && !product_ok(g_a, g_b))
+    return fail(NVFP4_EINVAL, "g_a and g_b must be finite with a finite product");
+  GemmParams p;
+  GemmTensorMaps maps;
+  GemmConfig cg;
+  const DeviceInfo* dev = nullptr;
+  nvfp4_status st = gemm_common(a, sfa, b, sfb, M, N, K, g_b, bias, &p, &maps, &cg, &dev, false, false, false, y);
+  if (st != NVFP4_OK) return st;
+  p.alpha_mul = g_a;
+  p.alpha_scale = g_a_device;
+  p.amax_out = reinterpret_cast<unsigned*>(amax_out);
+  st = make_tmap(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, M, N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B, "Y");
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_gemm(maps, p, cg, false, false, static_cast<cudaStream_t>(stream), *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return ok();
+}
 
 nvfp4_status nvfp4_gemm_quant(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb,
                               int64_t M, int64_t N, int64_t K, float alpha, const void* bias,

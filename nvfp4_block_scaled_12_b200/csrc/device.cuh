@@ -84,6 +84,19 @@ __device__ __forceinline__ uint32_t quantize_block16(const float (&v)[16], float
   return s;
 }
 
+// The per-tensor scale a measured amax gives (the dynamic quantizer's rule):
+// g = fl(amax / 2688) clamped into [2^-64, 2^64], 0 for amax == 0.
+__device__ __forceinline__ float scale_from_amax(float amax) {
+  return amax > 0.0f ? fminf(fmaxf(__fdiv_rn(amax, 2688.0f), 0x1p-64f), 0x1p64f) : 0.0f;
+}
+
+// Largest magnitude of the 2 x 16 bf16 values in a word, folded into acc (two
+// 16-bit lanes): |v| as its bit pattern orders like the value; a NaN counts
+// as infinity.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t acc, uint32_t w) {
+  return __vmaxu2(acc, __vminu2(w & 0x7FFF7FFFu, 0x7F807F80u));
+}
+
 // MXFP8 block (OCP microscaling): 32 fp32 values (exactly representable in
 // bf16) -> 32 E4M3 bytes in 8 little-endian words and the E8M0 scale byte.
 //   amax == 0: scale byte 0 (2^-127);  else s = clamp(floor(log2 amax) - 8,

@@ -646,6 +646,16 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
   // (pend holds the codes of a 64-column group's first chunk until its second
   // one completes the row's 32 bytes, written as one whole sector)
   const bool codes32 = (reinterpret_cast<uintptr_t>(p.codes_next) & 31u) == 0;
+  // plain epilogue with an amax output: this thread's largest |Y| so far (two
+  // bf16 lanes), folded into p.amax_out once per warp when its role ends
+  const bool want_amax = !kFused && p.amax_out != nullptr;
+  uint32_t amax2 = 0u;
+  auto flush_amax = [&]() {
+    if (!want_amax) return;
+    __syncwarp();
+    const uint32_t m = __reduce_max_sync(0xffffffffu, max(amax2 & 0xFFFFu, amax2 >> 16));
+    if (lane == 0 && m != 0u) atomicMax(p.amax_out, m << 16);  // the bf16 bits as float bits
+  };
   auto emit_chunk = [&](uint32_t (&w)[16], int n, int row_base, uint8_t* stage_buf, int& buf, uint32_t& sf_word,
                         uint32_t (&pend)[4]) {
     const int row = row_base + lane;
@@ -667,6 +677,10 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
     if (!kFused || dst == NVFP4_DST_BF16) {
       if (row_base < p.M) {
         store_chunk_bf16(&tmap_y, stage_buf + buf * 2048, w, lane, out_col, row_base);
+        if (want_amax && row < p.M) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) amax2 = bf16x2_absmax(amax2, w[j]);
+        }
         buf ^= 1;
       }
     } else {
@@ -793,6 +807,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         emit_chunk(w, n, row_base, stage_buf, buf, sf_word, pend);
       }
     }
+    flush_amax();
     if (lane == 0) bulk_wait<0>();
     if (fault != 0u) *abort_flag = 1;
     }
@@ -893,6 +908,7 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         acc_phase ^= 1u;
       }
     }
+    flush_amax();
     if (lane == 0) bulk_wait<0>();
     if (fault != 0u) *abort_flag = 1;
     }
@@ -971,7 +987,9 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
                                    pack_bf16x2(fmaf(alpha, v[4], bf16_lo(bv.z)), fmaf(alpha, v[5], bf16_hi(bv.z))),
                                    pack_bf16x2(fmaf(alpha, v[6], bf16_lo(bv.w)), fmaf(alpha, v[7], bf16_hi(bv.w))));
         *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(m) * p.ldy + n) = o;
+        if (want_amax) amax2 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(amax2, o.x), o.y), o.z), o.w);
       }
+      flush_amax();
     }
   }
   if (fault != 0u && lane == 0 && p.fault != nullptr) atomicOr(p.fault, fault);

@@ -41,6 +41,7 @@ struct GemmParams {
   __nv_bfloat16* y;           // K split: the bf16 output [M, ldy], written by the cluster's reduction
   int32_t ldy;
   const __nv_bfloat16* bias;  // nullable
+  unsigned* amax_out;         // nullable (plain epilogue): atomic max of |Y| as float bits
   unsigned* fault;
   // fused epilogue (only read by the fused kernel)
   int32_t n_ranges;
@@ -65,6 +66,7 @@ struct DynamicScaleArgs {
   float* scale_out;  // [0] amax, [1] g, written by CTA 0
   uint64_t wait_limit_ns;  // longest wait for the other CTAs' arrivals
   uint32_t expect;         // arrivals that complete the wait (the grid size, plus any test-only extra)
+  const float* amax_in;    // one-pass variant: g derived on the device from this amax (no amax pass)
 };
 
 // Grid-wait settings of the dynamic quantize (normally kWaitLimitNs and no
@@ -85,6 +87,11 @@ cudaError_t launch_quantize(const CUtensorMap& tmap_x, int tile_rows, int64_t M,
 // MXFP8 (E4M3 codes [M, K], E8M0 scales, one per 32 elements, swizzled).
 cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, uint8_t* codes,
                                   uint8_t* sf, cudaStream_t stream, const DeviceInfo& dev);
+// Same, with g derived on the device from amax_in[0] (as the dynamic
+// variant derives it from its own amax pass); scale_out gets [amax, g].
+cudaError_t launch_quantize_from_amax(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K,
+                                      const float* amax_in, uint8_t* codes, uint8_t* sf, float* scale_out,
+                                      cudaStream_t stream, const DeviceInfo& dev);
 // Same, with g measured on x in the same (cooperative) launch.
 cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, int tile_rows, const void* x, int64_t M, int64_t K,
                                     uint8_t* codes, uint8_t* sf, float* scale_out, uint32_t* scratch,

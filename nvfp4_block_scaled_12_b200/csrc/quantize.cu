@@ -128,6 +128,15 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
     const int64_t m_padded = (M + 127) & ~int64_t(127);  // rows of the scale buffer
     float amax_part = 0.0f;         // dynamic: max |x| over the rows this thread saw
     bool have_scale = !kDynamic;
+    if (!kDynamic && dyn.amax_in != nullptr) {
+      // one-pass variant: the scale comes from an amax measured elsewhere
+      const float amax = *dyn.amax_in;
+      g = scale_from_amax(amax);
+      if (blockIdx.x == 0 && warp == 0 && lane == 0) {
+        dyn.scale_out[0] = amax;
+        dyn.scale_out[1] = g;
+      }
+    }
     float d6 = __fmul_rn(6.0f, g);
     const int64_t katoms = K >> 6;
     // 32-byte aligned codes rows (the usual case: every row starts at a
@@ -167,8 +176,7 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
         *abort_flag = 1;
         return false;
       }
-      // g = fl(amax / 2688) clamped into [2^-64, 2^64]; 0 for an all-zero tensor
-      g = amax > 0.0f ? fminf(fmaxf(__fdiv_rn(amax, 2688.0f), 0x1p-64f), 0x1p64f) : 0.0f;
+      g = scale_from_amax(amax);
       d6 = __fmul_rn(6.0f, g);
       if (blockIdx.x == 0 && warp == 0 && lane == 0) {
         dyn.scale_out[0] = amax;
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
           f[8 * h + 6] = bf16_lo(u.w);
           f[8 * h + 7] = bf16_hi(u.w);
         }
-        if (kDynamic && g == 0.0f) {  // all-zero tensor: zero codes and scales
+        if (g == 0.0f) {  // measured scale of an all-zero tensor: zero codes and scales
           cw[2 * b] = 0u;
           cw[2 * b + 1] = 0u;
         } else {
@@ -381,6 +389,22 @@ cudaError_t launch_q(const CUtensorMap& tmap_x, const void* x, int64_t M, int64_
   return cudaGetLastError();
 }
 
+// The one-pass quantize with g from a device amax: the static kernel's grid.
+template <int kRows>
+cudaError_t launch_q_amax(const CUtensorMap& tmap_x, int64_t M, int64_t K, uint8_t* codes, uint8_t* sf,
+                          const DynamicScaleArgs& dyn, cudaStream_t stream, const DeviceInfo& dev) {
+  using Q = QCfg<kRows>;
+  const int64_t tiles_m = (M + kRows - 1) / kRows;
+  const int64_t tiles_k = (K + Q::kCols - 1) / Q::kCols;
+  const int64_t n_tiles = tiles_m * tiles_k;
+  const int grid = static_cast<int>(n_tiles < dev.num_sms ? n_tiles : dev.num_sms);
+  auto kernel = quantize_kernel<false, false, kRows>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Q::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  kernel<<<grid, Q::kThreads, Q::kSmemBytes, stream>>>(tmap_x, M, K, 0.0f, codes, sf, tiles_k, n_tiles, dev.fault, dyn);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K, float g, uint8_t* codes,
@@ -395,6 +419,16 @@ cudaError_t launch_quantize_mxfp8(const CUtensorMap& tmap_x, int tile_rows, int6
   const GridWaitSettings none;
   return tile_rows == 256 ? launch_q<false, true, 256>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, none, stream, dev)
                           : launch_q<false, true, 128>(tmap_x, nullptr, M, K, 0.0f, codes, sf, nullptr, nullptr, none, stream, dev);
+}
+
+cudaError_t launch_quantize_from_amax(const CUtensorMap& tmap_x, int tile_rows, int64_t M, int64_t K,
+                                      const float* amax_in, uint8_t* codes, uint8_t* sf, float* scale_out,
+                                      cudaStream_t stream, const DeviceInfo& dev) {
+  DynamicScaleArgs dyn{};
+  dyn.scale_out = scale_out;
+  dyn.amax_in = amax_in;
+  return tile_rows == 256 ? launch_q_amax<256>(tmap_x, M, K, codes, sf, dyn, stream, dev)
+                          : launch_q_amax<128>(tmap_x, M, K, codes, sf, dyn, stream, dev);
 }
 
 cudaError_t launch_quantize_dynamic(const CUtensorMap& tmap_x, int tile_rows, const void* x, int64_t M, int64_t K,

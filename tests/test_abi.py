@@ -24,7 +24,8 @@ def test_header_declares_the_expected_entry_points():
     for n in ("nvfp4_sf_bytes", "nvfp4_calibrate", "nvfp4_quantize", "nvfp4_swizzle_sf", "nvfp4_gemm",
               "nvfp4_gemm_quant", "nvfp4_quantize_dynamic", "nvfp4_gemm_dynamic", "nvfp4_mxfp8_sf_bytes",
               "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize", "nvfp4_fp8row_gemm",
-              "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_last_error"):
+              "nvfp4_dequantize", "nvfp4_check_fault", "nvfp4_last_error", "nvfp4_gemm_amax",
+              "nvfp4_quantize_from_amax"):
         assert n in names
 
 
@@ -100,6 +101,26 @@ def test_dynamic_entry_points_reject_bad_arguments_on_the_host():
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, 1.0, 0, 0, P, 0)   # no g_a
     _expect(F.NVFP4_EALIGN, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, 1.0, P + 1, 0, P, 0)
     _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_dynamic, P, P, P, P, 16, 64, 64, float("nan"), P, 0, P, 0)
+
+
+def test_amax_entry_points_reject_bad_arguments_on_the_host():
+    # nvfp4_gemm_amax(a, sfa, b, sfb, M, N, K, g_a, g_a_device, g_b, bias, y, amax_out, stream)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, 1.0, 0, 1.0, 0, P, 0, 0)    # no amax_out
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, 1.0, 0, 1.0, 0, 0, P, 0)    # no y
+    _expect(F.NVFP4_EALIGN, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, 1.0, 0, 1.0, 0, P, P + 2, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, 1.0, P + 1, 1.0, 0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, float("inf"), 0, 1.0, 0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, 3e38, 0, 10.0, 0, P, P, 0)  # product
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_amax, P, P, P, P, 16, 64, 64, 1.0, P, float("nan"), 0, P, P, 0)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_gemm_amax, P, P, P, P, 16, 12, 64, 1.0, 0, 1.0, 0, P, P, 0)    # N % 8
+    # nvfp4_quantize_from_amax(x, M, K, amax, codes, sf, scale_out, stream)
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_from_amax, P, 4, 64, 0, P, P, P, 0)      # no amax
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_from_amax, P, 4, 64, P, P, P, 0, 0)      # no scale_out
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_from_amax, P, 4, 96, P, P, P, P, 0)      # K % 64
+    _expect(F.NVFP4_EINVAL, F.nvfp4_quantize_from_amax, P, 0, 64, P, P, P, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_quantize_from_amax, P + 8, 4, 64, P, P, P, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_quantize_from_amax, P, 4, 64, P + 2, P, P, P, 0)
+    _expect(F.NVFP4_EALIGN, F.nvfp4_quantize_from_amax, P, 4, 64, P, P, P, P + 1, 0)
 
 
 @pytest.mark.parametrize("rows,k,want", [(4608, 3072, 4608 * 96), (1, 64, 128 * 4), (129, 192, 256 * 8),

@@ -38,7 +38,7 @@ def calls(monkeypatch):
     rec = []
     for name in ("nvfp4_quantize", "nvfp4_quantize_dynamic", "nvfp4_gemm", "nvfp4_gemm_dynamic",
                  "nvfp4_gemm_scaled", "nvfp4_gemm_quant_scaled", "nvfp4_gemm_quant", "nvfp4_mxfp8_quantize", "nvfp4_mxfp8_gemm", "nvfp4_fp8row_quantize",
-                 "nvfp4_fp8row_gemm", "nvfp4_dequantize"):
+                 "nvfp4_fp8row_gemm", "nvfp4_dequantize", "nvfp4_gemm_amax", "nvfp4_quantize_from_amax"):
         monkeypatch.setattr(F, name, lambda *a, _n=name: rec.append(_n))
     monkeypatch.setattr(F, "_stream", lambda stream: 0)
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
@@ -113,3 +113,23 @@ def test_malformed_outputs_are_rejected_before_the_call(calls):
                       F.FP8RowTensor(empty(N, K), empty(N, dtype=torch.float32), N, K),
                       y=empty(M, N - 8, dtype=torch.bfloat16))
     assert calls == []
+
+
+def test_amax_helpers_check_their_buffers(calls):
+    M, N, K = 130, 192, 256
+    x = empty(M, K, dtype=torch.bfloat16)
+    a, b = nvfp4(M, K), nvfp4(N, K)
+    amax = empty(1, dtype=torch.float32)
+    y = empty(M, N, dtype=torch.bfloat16)
+    d = F.NVFP4Tensor(empty(M, K // 2), empty(F.nvfp4_sf_bytes(M, K)), None, M, K, empty(2, dtype=torch.float32))
+    F.gemm(a, b, y=y, amax_out=amax)
+    F.gemm(a, b, alpha=0.5, y=y, amax_out=amax)
+    F.quantize_from_amax(x, amax, out=d)
+    assert calls == ["nvfp4_gemm_amax", "nvfp4_gemm_amax", "nvfp4_quantize_from_amax"]
+    with pytest.raises((TypeError, ValueError)):
+        F.gemm(a, b, y=y, amax_out=empty(1, dtype=torch.float16))
+    with pytest.raises((TypeError, ValueError)):
+        F.quantize_from_amax(x, empty(1, dtype=torch.int32), out=d)
+    with pytest.raises((TypeError, ValueError)):
+        F.quantize_from_amax(x, amax, out=F.NVFP4Tensor(empty(M, K // 2), empty(F.nvfp4_sf_bytes(M, K)), None,
+                                                        M, K, empty(1, dtype=torch.float32)))
