@@ -498,7 +498,7 @@ nvfp4_status nvfp4_gemm_tile_shape(int64_t M, int64_t N, int32_t num_sms, int32_
 
 /*
  * Launch plan of the GEMMs with the plain epilogue -- nvfp4_gemm,
- * nvfp4_gemm_scaled, nvfp4_gemm_dynamic (w4a16 = 0) and nvfp4_w4a16_gemm
+ * nvfp4_gemm_scaled, nvfp4_gemm_dynamic, nvfp4_gemm_amax (w4a16 = 0) and nvfp4_w4a16_gemm
  * (w4a16 = 1) -- for an M x N x K problem on num_sms SMs (host only):
  *   out[0..2] = tile shape as nvfp4_gemm_tile_shape reports it,
  *   out[3]    = K split: tile groups (CTAs or CTA pairs) that share one
