@@ -84,6 +84,46 @@ __device__ __forceinline__ uint32_t quantize_block16(const float (&v)[16], float
   return s;
 }
 
+// E4M3_satfinite(fl(amax / d6)) without the IEEE division's range check and
+// slow-path branch, given rd6 = RN(1/d6) and amax >= 0: q1 = fl(amax rd6) is
+// within 1.5 ulp of the quotient; at 1024 or more the quotient is far above
+// E4M3's largest value 448 and the code saturates; otherwise two FMA residual
+// corrections make it the correctly rounded quotient (Markstein, IBM J. Res.
+// Dev. 34(1), 1990: with rd6 the correctly rounded reciprocal and a faithful
+// q, RN(q + rd6 (amax - d6 q)) = RN(amax / d6)).  For d6 = fl(6 g), g in
+// [2^-64, 2^64], every residual of a quotient >= 2^-12 is exact; below that
+// the code is zero either way.
+__device__ __forceinline__ uint32_t block_scale_e4m3(float amax, float d6, float rd6) {
+  const float q1 = __fmul_rn(amax, rd6);
+  if (q1 >= 1024.0f) return 0x7Eu;  // 448
+  const float q2 = __fmaf_rn(__fmaf_rn(-q1, d6, amax), rd6, q1);
+  const float q3 = __fmaf_rn(__fmaf_rn(-q2, d6, amax), rd6, q2);
+  return e4m3_from_f32_satfinite(q3);
+}
+
+// quantize_block16 for the standalone quantizer: the block scale from
+// block_scale_e4m3, and the block's reciprocal from a table filled once per
+// launch, rtab[s] = RN(1 / fl(e4m3(s) g)) for the codes s = 1 .. 126 --
+// the same fp32 operations, taken out of the per-block path.
+__device__ __forceinline__ uint32_t quantize_block16_tab(const float (&v)[16], float d6, float rd6,
+                                                         const float* rtab, uint32_t& lo_word, uint32_t& hi_word) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t s = block_scale_e4m3(amax, d6, rd6);
+  lo_word = 0u;
+  hi_word = 0u;
+  if (s != 0u) {
+    const float r = rtab[s];
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], r);
+    lo_word = e2m1x8_from_f32(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+    hi_word = e2m1x8_from_f32(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+  }
+  return s;
+}
+
 // The per-tensor scale a measured amax gives (the dynamic quantizer's rule):
 // g = fl(amax / 2688) clamped into [2^-64, 2^64], 0 for amax == 0.
 __device__ __forceinline__ float scale_from_amax(float amax) {

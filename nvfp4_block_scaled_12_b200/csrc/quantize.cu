@@ -49,7 +49,8 @@ struct QCfg {
   static constexpr uint32_t kTileBytes = kRows * kCols * 2;
   static constexpr uint32_t kOffBar = kStages * kTileBytes;
   static constexpr uint32_t kOffMax = kOffBar + 2 * kStages * 8 + 16;  // per-warp maxima of the amax pass
-  static constexpr uint32_t kSmemBytes = kOffMax + (kConsumerWarps + 1) * 4 + 1024;  // + alignment slack
+  static constexpr uint32_t kOffRtab = (kOffMax + (kConsumerWarps + 1) * 4 + 15) & ~15u;  // 128 block reciprocals
+  static constexpr uint32_t kSmemBytes = kOffRtab + 128 * 4 + 1024;  // + alignment slack
   static_assert(kRows == 128 || kRows == 256, "tile rows");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -128,6 +129,14 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
     const int64_t m_padded = (M + 127) & ~int64_t(127);  // rows of the scale buffer
     float amax_part = 0.0f;         // dynamic: max |x| over the rows this thread saw
     bool have_scale = !kDynamic;
+    // rtab[s] = RN(1 / fl(e4m3(s) g)): the block reciprocal for every scale
+    // code, filled by the consumers once g is known
+    float* rtab = reinterpret_cast<float*>(smem + Q::kOffRtab);
+    auto fill_rtab = [&]() {
+      const int ct = warp * 32 + lane;
+      if (ct < 128) rtab[ct] = (ct >= 1 && ct <= 126) ? __frcp_rn(__fmul_rn(e4m3_to_f32(ct), g)) : 0.0f;
+      named_barrier_sync(1, Q::kConsumerWarps * 32);
+    };
     if (!kDynamic && dyn.amax_in != nullptr) {
       // one-pass variant: the scale comes from an amax measured elsewhere
       const float amax = *dyn.amax_in;
@@ -138,6 +147,8 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
       }
     }
     float d6 = __fmul_rn(6.0f, g);
+    float rd6 = __frcp_rn(d6);
+    if (!kDynamic && !kMx) fill_rtab();
     const int64_t katoms = K >> 6;
     // 32-byte aligned codes rows (the usual case: every row starts at a
     // multiple of 32 bytes when the buffer does) take one 32-byte store
@@ -178,6 +189,8 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
       }
       g = scale_from_amax(amax);
       d6 = __fmul_rn(6.0f, g);
+      rd6 = __frcp_rn(d6);
+      fill_rtab();
       if (blockIdx.x == 0 && warp == 0 && lane == 0) {
         dyn.scale_out[0] = amax;
         dyn.scale_out[1] = g;
@@ -293,7 +306,7 @@ __global__ void __launch_bounds__(QCfg<kRows>::kThreads, 1)
           cw[2 * b] = 0u;
           cw[2 * b + 1] = 0u;
         } else {
-          sfw |= quantize_block16(f, g, d6, cw[2 * b], cw[2 * b + 1]) << (8 * b);
+          sfw |= quantize_block16_tab(f, d6, rd6, rtab, cw[2 * b], cw[2 * b + 1]) << (8 * b);
         }
       }
       if (row < M) {
