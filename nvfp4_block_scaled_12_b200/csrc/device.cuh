@@ -61,29 +61,6 @@ __device__ __forceinline__ uint32_t e2m1x8_from_f32(float v0, float v1, float v2
   return out;
 }
 
-// Quantize 16 fp32 values (exactly representable in bf16) that form one
-// NVFP4 block, given the per-tensor scale g and d6 = fl(6*g).  Writes the 8
-// code bytes as two 32-bit words (element 0 in the low nibble of byte 0 of
-// lo_word) and returns the E4M3 scale byte.
-__device__ __forceinline__ uint32_t quantize_block16(const float (&v)[16], float g, float d6,
-                                                     uint32_t& lo_word, uint32_t& hi_word) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const uint32_t s = e4m3_from_f32_satfinite(__fdiv_rn(amax, d6));
-  lo_word = 0u;
-  hi_word = 0u;
-  if (s != 0u) {
-    const float r = __frcp_rn(__fmul_rn(e4m3_to_f32(s), g));
-    float q[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], r);
-    lo_word = e2m1x8_from_f32(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-    hi_word = e2m1x8_from_f32(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-  }
-  return s;
-}
-
 // E4M3_satfinite(fl(amax / d6)) without the IEEE division's range check and
 // slow-path branch, given rd6 = RN(1/d6) and amax >= 0: q1 = fl(amax rd6) is
 // within 1.5 ulp of the quotient; at 1024 or more the quotient is far above
@@ -101,10 +78,35 @@ __device__ __forceinline__ uint32_t block_scale_e4m3(float amax, float d6, float
   return e4m3_from_f32_satfinite(q3);
 }
 
-// quantize_block16 for the standalone quantizer: the block scale from
-// block_scale_e4m3, and the block's reciprocal from a table filled once per
-// launch, rtab[s] = RN(1 / fl(e4m3(s) g)) for the codes s = 1 .. 126 --
-// the same fp32 operations, taken out of the per-block path.
+// Quantize 16 fp32 values (exactly representable in bf16) that form one
+// NVFP4 block, given the per-tensor scale g, d6 = fl(6*g) and rd6 = RN(1/d6):
+//     s = E4M3_satfinite(fl(amax / d6))   (block_scale_e4m3)
+//     code_i = E2M1_satfinite(fl(v_i * RN(1 / fl(e4m3(s) * g))))   (0 when s == 0)
+// Writes the 8 code bytes as two 32-bit words (element 0 in the low nibble
+// of byte 0 of lo_word) and returns the E4M3 scale byte.
+__device__ __forceinline__ uint32_t quantize_block16_rd(const float (&v)[16], float g, float d6, float rd6,
+                                                        uint32_t& lo_word, uint32_t& hi_word) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t s = block_scale_e4m3(amax, d6, rd6);
+  lo_word = 0u;
+  hi_word = 0u;
+  if (s != 0u) {
+    const float r = __frcp_rn(__fmul_rn(e4m3_to_f32(s), g));
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], r);
+    lo_word = e2m1x8_from_f32(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+    hi_word = e2m1x8_from_f32(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+  }
+  return s;
+}
+
+// quantize_block16_rd for the standalone quantizer, with the block's
+// reciprocal from a table filled once per launch, rtab[s] = RN(1 / fl(e4m3(s)
+// g)) for the codes s = 1 .. 126: the same fp32 operations, taken out of the
+// per-block path.
 __device__ __forceinline__ uint32_t quantize_block16_tab(const float (&v)[16], float d6, float rd6,
                                                          const float* rtab, uint32_t& lo_word, uint32_t& hi_word) {
   float amax = 0.0f;

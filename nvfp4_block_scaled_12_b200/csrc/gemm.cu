@@ -646,6 +646,9 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
   // (pend holds the codes of a 64-column group's first chunk until its second
   // one completes the row's 32 bytes, written as one whole sector)
   const bool codes32 = (reinterpret_cast<uintptr_t>(p.codes_next) & 31u) == 0;
+  // the fused epilogue's quantize: d6 = fl(6 g_next) and its reciprocal, once
+  const float next_d6 = __fmul_rn(6.0f, p.g_next);
+  const float next_rd6 = __frcp_rn(next_d6);
   // plain epilogue with an amax output: this thread's largest |Y| so far (two
   // bf16 lanes), folded into p.amax_out once per warp when its role ends
   const bool want_amax = !kFused && p.amax_out != nullptr;
@@ -686,7 +689,6 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
     } else {
       // next layer's NVFP4 input: two 16-element blocks per chunk
       const float g = p.g_next;
-      const float d6 = __fmul_rn(6.0f, g);
       float blk[16];
       uint32_t c0, c1, c2, c3;
 #pragma unroll
@@ -694,13 +696,13 @@ __global__ void __launch_bounds__(Cfg<kCG, kBN, kAcc, kMx, kRow, kW16>::kThreads
         blk[2 * j] = bf16_lo(w[j]);
         blk[2 * j + 1] = bf16_hi(w[j]);
       }
-      const uint32_t s0 = quantize_block16(blk, g, d6, c0, c1);
+      const uint32_t s0 = quantize_block16_rd(blk, g, next_d6, next_rd6, c0, c1);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         blk[2 * j] = bf16_lo(w[8 + j]);
         blk[2 * j + 1] = bf16_hi(w[8 + j]);
       }
-      const uint32_t s1 = quantize_block16(blk, g, d6, c2, c3);
+      const uint32_t s1 = quantize_block16_rd(blk, g, next_d6, next_rd6, c2, c3);
       const int csf = out_col >> 4;  // scale column of the first block (even)
       uint8_t* crow = p.codes_next + static_cast<size_t>(row) * (p.k_next >> 1) + (out_col >> 1);
       if ((csf & 3) == 0) {
