@@ -261,10 +261,11 @@ nvfp4_status nvfp4_gemm_dynamic(const uint8_t* a, const uint8_t* sfa, const uint
 
 /*
  * The GEMM of nvfp4_gemm_scaled / nvfp4_gemm_dynamic that also measures its
- * output for the next layer's dynamic scale (the survey's "amax emitted by the
- * previous layer's epilogue": the next layer then quantizes in one pass with
- * nvfp4_quantize_from_amax instead of the two passes of
- * nvfp4_quantize_dynamic).
+ * output for the next layer's dynamic scale (a measured activation scale in
+ * place of the calibrated input_scale, "BFL (fp8r / nvfp4)" doc, nvfp4
+ * bullet, with the amax taken by the previous layer's epilogue: the next
+ * layer then quantizes in one pass with nvfp4_quantize_from_amax instead of
+ * the two passes of nvfp4_quantize_dynamic).
  *     Y = bf16( fl(g * g_b) * acc + bias ),  g = g_a_device ? g_a_device[0] : g_a
  *     amax_out[0] = max(amax_out[0], max |Y[m, n]|)  over the M x N outputs
  * The maximum is taken over the bf16 values written (a NaN counts as +inf)

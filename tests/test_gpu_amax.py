@@ -3,10 +3,10 @@ max|Y| of its own output (nvfp4_gemm_amax) and the quantizer that derives
 the per-tensor scale from a given amax on the device
 (nvfp4_quantize_from_amax).
 
-The survey's first "next" row lists this as the alternative to the two-pass
-dynamic quantize: the amax of a layer's input is emitted by the previous
-layer's epilogue ("BFL (fp8r / nvfp4)" doc, ``nvfp4`` bullet: the measured
-scale is the variant of the calibrated ``input_scale``).  The amax must equal
+This is the one-pass alternative to the two-pass dynamic quantize: the amax
+of a layer's input is emitted by the previous layer's epilogue ("BFL (fp8r /
+nvfp4)" doc, ``nvfp4`` bullet: the measured scale is the variant of the
+calibrated ``input_scale``).  The amax must equal
 the largest magnitude of the bf16 values the GEMM wrote, bit for bit, and the
 GEMM's Y must not change; the one-pass quantize must give the oracle's codes,
 scales, amax and g bit for bit, i.e. the same bytes as the two-pass dynamic
