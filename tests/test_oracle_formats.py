@@ -119,3 +119,21 @@ def test_round_to_bf16_matches_torch_on_fp32_inputs():
     ref = torch.from_numpy(f).to(torch.bfloat16).to(torch.float64).numpy()
     got = O.round_to_bf16(f.astype(np.float64))
     assert np.array_equal(got, ref)
+
+
+def test_code_packing_is_a_little_endian_stream_of_4_bit_fields():
+    # Two E2M1 codes per byte ("BFL (fp8r / nvfp4)" doc, nvfp4 bullet), the
+    # even element in the low nibble: the row's codes laid end to end as
+    # 4-bit little-endian fields, element 0 first, and cut into bytes.
+    # Built here from numpy's bit packing, not from the oracle's shifts.
+    rng = np.random.default_rng(7)
+    q = rng.integers(0, 16, (5, 64)).astype(np.uint8)
+    bits = ((q[:, :, None] >> np.arange(4, dtype=np.uint8)) & 1).reshape(5, 64 * 4)
+    want = np.packbits(bits, axis=1, bitorder="little")
+    got = O.pack_codes(q)
+    assert got.shape == (5, 32) and np.array_equal(got, want)
+    assert np.array_equal(O.unpack_codes(got), q)
+    # and every byte is the packing of exactly one code pair
+    b = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    assert np.array_equal(O.pack_codes(O.unpack_codes(b)), b)
+    assert O.pack_codes(np.array([[0x1, 0x2]], np.uint8))[0, 0] == 0x21

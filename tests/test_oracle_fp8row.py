@@ -79,3 +79,28 @@ def test_gemm_matches_a_triple_loop():
         for n in range(Nn):
             acc = sum(float(a[m, k:k + 1].view(F8)[0]) * float(b[n, k:k + 1].view(F8)[0]) for k in range(K))
             assert y[m, n] == pytest.approx(float(sa[m]) * float(sb[n]) * acc + bias[n], rel=1e-12, abs=1e-300)
+
+
+def test_dequantize_is_the_e4m3_value_times_the_row_scale():
+    # every non-NaN byte against ml_dtypes' E4M3, times an fp32 row scale, in
+    # exact float64 arithmetic
+    codes = np.arange(256, dtype=np.uint8)
+    codes = codes[(codes & 0x7F) != 0x7F].reshape(2, 127)
+    s = np.array([0.75, 2.0 ** -20], np.float32)
+    got = R.dequantize_fp8_rowwise(codes, s)
+    want = codes.view(F8).astype(np.float64) * s.astype(np.float64)[:, None]
+    assert np.array_equal(got, want)
+
+
+def test_representable_rows_round_trip():
+    # rows of E4M3 values times a power of two, with the top code present:
+    # s is that power of two and quantize -> dequantize gives the row back
+    rng = np.random.default_rng(44)
+    vals = N.e4m3_decode(np.arange(256, dtype=np.uint8))
+    vals = vals[~np.isnan(vals)]
+    for k in (-12, 0, 7):
+        x = (rng.choice(vals, (4, 96)) * 2.0 ** k).astype(np.float32)
+        x[:, 0] = 448.0 * 2.0 ** k
+        codes, s = R.quantize_fp8_rowwise(x)
+        assert np.all(s == np.float32(2.0 ** k))
+        assert np.array_equal(R.dequantize_fp8_rowwise(codes, s), x.astype(np.float64))

@@ -144,3 +144,20 @@ def test_gemm_matches_a_brute_force_triple_loop():
                 bv = float(b_codes[n, k:k + 1].view(F8)[0]) * 2.0 ** (int(b_sf[n, k // 32]) - 127)
                 acc += av * bv
             assert y[m, n] == pytest.approx(0.5 * acc + bias[n], rel=1e-12, abs=1e-300)
+
+
+def test_block_exponent_is_floor_log2_in_exact_arithmetic():
+    # 2^e <= a < 2^(e+1), checked with exact rationals, on powers of two and
+    # their neighbours, random normals, and fp32 subnormals
+    from fractions import Fraction
+    rng = np.random.default_rng(45)
+    a = [np.float32(2.0 ** e) for e in range(-149, 128)]
+    a += [np.nextafter(v, np.float32(0)) for v in a[1:]] + [np.nextafter(v, np.float32(np.inf)) for v in a[:-1]]
+    a += list(rng.uniform(1, 2, 300).astype(np.float32) * np.float32(2.0) ** rng.integers(-126, 127, 300))
+    a += list((rng.integers(1, 1 << 23, 100).astype(np.uint32)).view(np.float32))   # subnormals
+    a = np.array(a, np.float32)
+    a = a[np.isfinite(a) & (a > 0)]
+    e = X.block_exponent(a)
+    for v, k in zip(a, e):
+        f = Fraction(float(v))
+        assert Fraction(2) ** int(k) <= f < Fraction(2) ** (int(k) + 1), (v, k)
